@@ -1,0 +1,434 @@
+"""Benchmark of the sampled-softmax CE LM head (candidate build + forward + backward).
+
+One step = ss_build_candidates + ss_ce_forward + ss_ce_backward on one
+microbatch of the stage-2-late workload (T=49152 tokens, d=768, V=50304,
+P=24576), inputs resident in HBM. Metric: tokens/s over all ranks; the
+dense-contraction work of a step is 6*T*d*P FLOPs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the float64 CPU oracle, bounded sample
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own
+microbatch (seed + rank, negative-window offset staggered by V*rank/N); the
+path has no collective, so this is weak scaling, timed as the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sampled_softmax_cross_b200 import workloads as wl  # noqa: E402
+
+METRIC = "tokens/s fused sampled-CE fwd+bwd at P=24576,d=768; % of BF16 tensor peak"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=wl.HEADLINE, choices=list(wl.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=256,
+                    help="rows of the workload the oracle processes per reference step")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"],
+                    sm_max=p.get("sm_max_mhz"), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, sm_max=1965.0, src="fallback")
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        """Start sampling; returns once the first sample has arrived (or after 10 s)."""
+        import threading
+        self.lines = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        first = threading.Event()
+
+        def reader():
+            for line in self.proc.stdout:
+                self.lines.append(line)
+                first.set()
+
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        first.wait(10.0)
+        self.n_before = len(self.lines)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        # samples taken while the timed region ran (the first one marks its start)
+        lines = self.lines[max(0, self.n_before - 1):]
+        rows = [r for r in csv.reader(io.StringIO("".join(lines))) if len(r) >= 9]
+        if not rows:
+            return None
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------- reference --
+
+def oracle_sample_step(x64, lm64, targets, w, rows):
+    """One bounded oracle step: full candidate build, then loss and gradients of `rows` rows."""
+    from oracle import sampled_ce as oc
+    cand, tpos, vpos, _ = oc.build_candidates(targets, w.V, w.P, w.offset)
+    w_c = oc.gather_rows(lm64, cand)
+    xs = x64[:rows]
+    loss, lse, _, n = oc.sampled_ce_forward(xs, w_c, tpos[:rows])
+    oc.sampled_ce_backward(1.0, xs, w_c, cand, tpos[:rows], lse, w.V)
+    return loss
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return  # rank 0 alone runs the CPU oracle
+    x_bits, lm_bits, targets = wl.workload_inputs(w)
+    x64, lm64 = wl.bits_to_f64(x_bits), wl.bits_to_f64(lm_bits)
+    rows = min(args.cpu_rows, w.T)
+    # keep the whole run within a few minutes: shrink the sample if one step is slow
+    t0 = time.perf_counter()
+    oracle_sample_step(x64, lm64, targets, w, rows)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    while time.perf_counter() - t0 > budget and rows > 32:
+        rows //= 2
+        t0 = time.perf_counter()
+        oracle_sample_step(x64, lm64, targets, w, rows)
+    for _ in range(args.warmup):
+        oracle_sample_step(x64, lm64, targets, w, rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(x64, lm64, targets, w, rows)
+    dt = time.perf_counter() - t0
+    value = rows * args.steps / dt
+    sample = (f"{rows} of {w.T} rows of {w.name} per step (full candidate build + loss and "
+              f"gradients of those rows), float64 numpy")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, n):
+    return {"workload": f"{w.name}: T={w.T} d={w.d} V={w.V} P={w.P} (per rank)",
+            "T": w.T, "d": w.d, "V": w.V, "P": w.P, "offset": w.offset, "zipf_s": w.zipf_s,
+            "ignored_frac": w.ignore_frac, "seed": w.seed,
+            "parallelism": f"dp{n} (independent microbatch per rank, no collective)",
+            "l2": "no explicit flush: each step streams >2 GB of bf16 logits through HBM (L2 126 MB)"}
+
+
+# ------------------------------------------------------------------ ours --
+
+def source_hash(*names):
+    h = hashlib.sha1()
+    for n in names:
+        with open(os.path.join(ROOT, "sampled_softmax_cross_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f).get(kernel)
+    except Exception:
+        return None, None
+    if not rec:
+        return None, None
+    if rec.get("source_hash") != source_hash(*rec.get("sources", [])):
+        return None, "stale"
+    return rec.get("bytes_per_launch_full_size"), rec.get("note")
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from sampled_softmax_cross_b200 import build_lib, capi
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        build_lib.build()
+    if world > 1:
+        dist.barrier()
+    capi.load()
+
+    # this rank's microbatch: own seed, staggered window start
+    x_bits, lm_bits, targets = wl.make_inputs(w.T, w.d, w.V, w.zipf_s, w.ignore_frac, w.seed + rank)
+    offset = (w.offset + (w.V * rank) // world) % w.V
+    x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    lm = torch.from_numpy(lm_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    t = torch.from_numpy(targets).to(dev)
+    ce = capi.SampledCE(w.T, w.d, w.V, w.P, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ce.step(t, x, lm, offset, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = ce.status()
+    if st[0] != 0 or st[8] != 0:
+        raise RuntimeError(f"device status {st}")
+
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    capi.ss_timing_reset()
+    capi.ss_timing_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    clk = clocks.stop()
+    capi.ss_timing_enable(False)
+    kernels = capi.ss_timing_read()
+    capi.ss_timing_reset()
+    launches = sum(n for n, _ in kernels.values())
+
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # e2e: the same step from pinned host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hx = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        hlm = torch.from_numpy(lm_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        ht = torch.from_numpy(targets).pin_memory()
+        hloss = torch.empty(1, dtype=torch.float32).pin_memory()
+        hdx = torch.empty((w.T, w.d), dtype=torch.bfloat16).pin_memory()
+        hdW = torch.empty((w.V, w.d), dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step():
+            x.copy_(hx, non_blocking=True)
+            lm.copy_(hlm, non_blocking=True)
+            t.copy_(ht, non_blocking=True)
+            step()
+            hloss.copy_(ce.loss, non_blocking=True)
+            hdx.copy_(ce.dx[: w.T], non_blocking=True)
+            hdW.copy_(ce.dW, non_blocking=True)
+
+        for _ in range(max(1, args.warmup // 2)):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        k2 = max(3, args.steps // 2)
+        for _ in range(k2):
+            e2e_step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = torch.tensor([ev0.elapsed_time(ev1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        h2d = hx.numel() * 2 + hlm.numel() * 2 + ht.numel() * 4
+        d2h = 4 + hdx.numel() * 2 + hdW.numel() * 2
+        e2e = {"value": w.T * world * k2 / (float(e_ms.item()) / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": float(e_ms.item()) / k2}
+
+    if rank == 0:
+        pk = peaks()
+        tokens = w.T * world * args.steps
+        value = tokens / (ms_max / 1e3)
+        per = {}
+        flops_gemm = 2.0 * w.T * w.d * w.P
+        alg = {  # algorithmic work per launch
+            "fwd_gemm_ce": ("tensor", flops_gemm), "dx_gemm": ("tensor", flops_gemm),
+            "dw_gemm_scatter": ("tensor", flops_gemm),
+            "gather": ("hbm", 2.0 * w.P * w.d * 2),
+            "dlogits": ("hbm", 2.0 * w.T * w.P * 2),
+            "zero_rows": ("hbm", (w.V - w.P) * w.d * 2.0 + w.V * 4),
+            "build_mark": ("hbm", w.T * 4.0 + 2 * ((w.V + 31) // 32) * 4),
+            "build_emit": ("hbm", w.T * 4.0 * 2 + w.V * 4.0 * 2 + w.P * 4.0),
+            "lse_combine": ("hbm", ((w.P + 255) // 256) * w.T * 8.0 + w.T * 16.0),
+        }
+        total_k = sum(t for _, t in kernels.values())
+        for k, (n, tot) in kernels.items():
+            avg = tot / max(n, 1)
+            e = {"launches": n, "avg_ms": avg, "share": tot / total_k if total_k else None}
+            if k in alg:
+                bound, work = alg[k]
+                if bound == "tensor":
+                    e["tflops"] = work / (avg / 1e3) / 1e12
+                    e["frac_of_sustained"] = e["tflops"] / pk["bf16_sus"]
+                else:
+                    e["gbs"] = work / (avg / 1e3) / 1e9
+                    e["frac_of_hbm"] = e["gbs"] / pk["hbm"]
+            per[k] = e
+        dom = max(kernels, key=lambda k: kernels[k][1])
+        bound, work = alg.get(dom, ("tensor", flops_gemm))
+        avg = kernels[dom][1] / kernels[dom][0]
+        traffic, tnote = traffic_for(dom)
+        if bound == "tensor":
+            ach = work / (avg / 1e3) / 1e12
+            roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": pk["bf16_sus"],
+                    "unit": "TFLOP/s", "frac": ach / pk["bf16_sus"],
+                    "peak_note": f"bf16 sustained ({pk['src']}); burst {pk['bf16']} gives frac "
+                                 f"{ach / pk['bf16']:.3f}",
+                    "traffic": traffic, "algorithmic_per_launch": work}
+        else:
+            ach = work / (avg / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": pk["hbm"],
+                    "unit": "GB/s", "frac": ach / pk["hbm"], "traffic": traffic,
+                    "algorithmic_per_launch": work}
+        if tnote:
+            roof["traffic_note"] = tnote
+        step_tflops = 6.0 * w.T * w.d * w.P * world * args.steps / (ms_max / 1e3) / 1e12
+
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            rows = min(512, w.T)
+            x64, lm64 = wl.bits_to_f64(x_bits), wl.bits_to_f64(lm_bits)
+            t0 = time.perf_counter()
+            reps = 0
+            while True:
+                oracle_sample_step(x64, lm64, targets, w, rows)
+                reps += 1
+                if time.perf_counter() - t0 > 8.0 or reps >= 8:
+                    break
+            dt = time.perf_counter() - t0
+            cpu = {"value": rows * reps / dt, "unit": "tokens/s", "cores": blas_threads(),
+                   "kind": "oracle",
+                   "sample": f"{reps} x ({rows} of {w.T} rows of {w.name}: full candidate build "
+                             f"+ float64 loss and gradients of those rows)"}
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Zipf targets, N(0,1) x, N(0,1/d) lm_head)",
+            "config": workload_config(w, world),
+            "step_tflops": step_tflops,
+            "frac_of_bf16_peak": {"sustained": step_tflops / pk["bf16_sus"],
+                                  "burst": step_tflops / pk["bf16"], "datasheet_2250": step_tflops / 2250.0,
+                                  "peaks": pk["src"]},
+            "roofline": roof,
+            "kernels": per,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

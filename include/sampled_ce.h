@@ -1,0 +1,170 @@
+/*
+ * sampled_ce.h -- C ABI of the B200 (sm_100a) shared-negatives sampled-softmax
+ * cross-entropy LM head: candidate build, forward and backward.
+ *
+ * The method is the one of "sampled_softmax.py" (modded-nanogpt,
+ * track_1_short): every token of a microbatch shares one candidate set C of
+ * P classes -- every class that is a target somewhere in the microbatch, plus
+ * negatives taken from the next window of the stride permutation
+ * k * stride mod V -- and the cross-entropy is a softmax over C instead of
+ * the whole vocabulary (module docstring, "What"). The lm_head gradient is
+ * dense over the vocabulary with zeros outside C.
+ *
+ * Conventions for every entry point
+ *   - All array arguments are DEVICE pointers on the current CUDA device,
+ *     row-major and contiguous, 16-byte aligned. bf16 values are passed as
+ *     their raw 16-bit patterns (ss_bf16).
+ *   - The caller owns every buffer, the workspace included. The library
+ *     allocates no device memory and keeps no state between calls, apart
+ *     from per-device launch attributes it sets once.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). All work
+ *     is enqueued on it; no call synchronises the device.
+ *   - Host-detectable errors (sizes, alignment, workspace too small, a
+ *     stride not coprime with V, a device that is not sm_100) return a
+ *     non-zero ss_status before anything is enqueued. Errors that only the
+ *     device can see are written to `dev_status` (below); read it after the
+ *     stream has reached the call.
+ *   - Index types are int32 (V < 2^31). The ignore marker for a target is -1.
+ *
+ * dev_status: int32[SS_DEV_STATUS_WORDS], device memory. ss_build_candidates
+ * rewrites all 16 words; ss_ce_forward and ss_ce_backward only ever set
+ * words 8..9 (first error wins), so one buffer can serve a whole step.
+ *   [0] builder status (ss_status)      [1] D: distinct valid targets
+ *   [2] need = P - D                    [3] 1 if the fallback pick ran
+ *   [4] draw: window positions consumed [5] next offset = (offset + draw) mod V
+ *   [6] first token index with a bad target, else -1
+ *   [7] number of classes marked (P when the build succeeded)
+ *   [8] forward/backward kernel error (ss_status, 0 = none)
+ *   [9] detail for [8] (kernel id)      [10..15] reserved (0)
+ */
+#ifndef SAMPLED_CE_H
+#define SAMPLED_CE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SS_API __attribute__((visibility("default")))
+#else
+#define SS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t ss_bf16; /* raw bfloat16 bits */
+
+typedef enum ss_status {
+  SS_OK = 0,
+  SS_ERR_INVALID_ARG = 1,        /* a size or pointer argument is out of range */
+  SS_ERR_BAD_TARGET = 2,         /* a target outside [-1, V) (device) */
+  SS_ERR_TOO_MANY_TARGETS = 3,   /* D > P distinct targets (device) */
+  SS_ERR_NO_FREE_CLASSES = 4,    /* fewer than P - D classes left (device) */
+  SS_ERR_STRIDE_NOT_COPRIME = 5, /* gcd(stride, V) != 1 */
+  SS_ERR_WORKSPACE_TOO_SMALL = 6,
+  SS_ERR_MISALIGNED = 7,         /* a pointer is not 16-byte aligned */
+  SS_ERR_CUDA = 8,               /* a CUDA runtime call failed; see ss_last_cuda_error */
+  SS_ERR_UNSUPPORTED_DEVICE = 9, /* the current device is not compute capability 10.x */
+  SS_ERR_KERNEL_TIMEOUT = 10,    /* a pipeline wait ran out of time (device) */
+  SS_ERR_BAD_INDEX = 11          /* a candidate or position outside its range (device) */
+} ss_status;
+
+#define SS_DEV_STATUS_WORDS 16
+#define SS_DEFAULT_STRIDE 20011 /* NEGATIVE_STRIDE of sampled_softmax.py */
+#define SS_MAX_VOCAB (1 << 19)  /* largest V the candidate builder accepts */
+
+/* Bytes of workspace the three calls need for these sizes (0 if the sizes
+ * are invalid). One workspace serves ss_build_candidates, ss_ce_forward and
+ * ss_ce_backward of the same microbatch; ss_ce_forward leaves the gathered
+ * rows W_C and the bf16 logits in it for ss_ce_backward, so it must not be
+ * reused between a forward and its backward (the "one microbatch per step"
+ * contract of sampled_softmax.py, SampledSoftmax.__init__). */
+SS_API size_t ss_workspace_bytes(int64_t T, int32_t d, int32_t V, int32_t P);
+
+/* Bytes of workspace ss_build_candidates alone needs for a vocabulary of V
+ * classes (0 if V is out of range). ss_workspace_bytes covers it as well. */
+SS_API size_t ss_build_workspace_bytes(int32_t V);
+
+/* Candidate set C for one microbatch.
+ * sampled_softmax.py, CandidateBuilder.build and CandidateBuilder._negatives:
+ *   mark every valid target; D = number of marked classes (D > P is an error);
+ *   if D < P take need = P - D negatives: the first `need` unmarked classes of
+ *   the stride sweep c_k = (stride * k) mod V for k = offset, offset+1, ...,
+ *   offset+draw-1 (k mod V), draw = min(V, floor(1.7 * need) + 256); if that
+ *   window holds fewer than `need` unmarked classes, take instead
+ *   free[0 :: max(1, |free| / need)][:need] over the ascending unmarked classes.
+ *   C = marked classes in ascending order.
+ * In:  targets [T] int32, each in [-1, V) (-1 = ignored token);
+ *      offset >= 0 (reduced mod V); stride coprime with V (SS_DEFAULT_STRIDE).
+ *      1 <= P <= V <= SS_MAX_VOCAB, T >= 0.
+ * Out: candidates [P] int32 ascending class ids;
+ *      target_pos [T] int32: position of targets[i] in C, -1 for ignored;
+ *      vocab_pos  [V] int32: position of each class in C, -1 outside C;
+ *      dev_status [16] (see above). On a device-detected error the three
+ *      arrays are filled with -1. */
+SS_API ss_status ss_build_candidates(const int32_t* targets, int64_t T, int32_t V, int32_t P,
+                              int64_t offset, int32_t stride, int32_t* candidates,
+                              int32_t* target_pos, int32_t* vocab_pos, int32_t* dev_status,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Forward: W_C = lm_head[C] (sampled_softmax.py, SampledSoftmax._gather_rows),
+ * logits z = x @ W_C^T with fp32 accumulation, and an online-softmax
+ * cross-entropy over the P columns ("Learning Triton One Kernel at a Time:
+ * Softmax", section "Online Softmax"):
+ *   lse[i]  = log sum_j exp(z_ij), for every row (ignored rows included);
+ *   loss    = sum over valid rows of (lse[i] - z[i, target_pos[i]]) / n_valid,
+ *             0 when n_valid = 0 (token-weighted mean, as in Handout #16's
+ *             lm_gradient);
+ *   n_valid = number of rows with target_pos >= 0.
+ * In:  x [T, d] bf16; lm_head [V, d] bf16; candidates [P], target_pos [T] as
+ *      written by ss_build_candidates. d % 8 == 0.
+ * Out: loss [1] float32, lse [T] float32, n_valid [1] int32.
+ * Workspace: keeps W_C [P, d] bf16 and the bf16 logits [T, P] for the backward. */
+SS_API ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t* candidates,
+                        const int32_t* target_pos, int64_t T, int32_t d, int32_t V, int32_t P,
+                        float* loss, float* lse, int32_t* n_valid, int32_t* dev_status,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of the loss above for an upstream gradient g = grad_loss[0]
+ * ("Learning Triton ... Softmax", section "Gradient": softmax minus one-hot):
+ *   G_ij  = (g / n_valid) * (exp(z_ij - lse_i) - [j == target_pos_i]), valid rows;
+ *   G_i   = 0 for ignored rows (and everywhere when n_valid = 0);
+ *   dx    = G @ W_C                      [T, d] bf16;
+ *   dW    = dense [V, d] bf16: row C_j = (G^T @ x)_j, every other row +0.0
+ *           (module docstring: "dense over the vocabulary with zeros outside C").
+ * In:  grad_loss [1] float32 (device); x, candidates, target_pos, vocab_pos as
+ *      above; lse and n_valid from ss_ce_forward; the workspace the forward used.
+ * Out: dx [T, d], dW [V, d] (fully written). The logits in the workspace are
+ *      overwritten with G. */
+SS_API ss_status ss_ce_backward(const float* grad_loss, const ss_bf16* x, const int32_t* candidates,
+                         const int32_t* target_pos, const int32_t* vocab_pos, const float* lse,
+                         const int32_t* n_valid, int64_t T, int32_t d, int32_t V, int32_t P,
+                         ss_bf16* dx, ss_bf16* dW, int32_t* dev_status, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+SS_API const char* ss_status_string(int32_t status);
+
+/* Text of the last CUDA runtime error seen by this thread ("" if none). */
+SS_API const char* ss_last_cuda_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+SS_API int32_t ss_version(void);
+
+/* Kernel timing for diagnostics. While enabled, each kernel launch the library
+ * makes is bracketed by two CUDA events recorded on its stream (a pool of
+ * 8192 launches; later launches go untimed). ss_timing_query synchronises on
+ * the recorded events and returns, for the i-th distinct kernel name, its
+ * launch count and total milliseconds. Not thread-safe; for benchmarks. */
+SS_API ss_status ss_timing_enable(int32_t enable);
+SS_API ss_status ss_timing_reset(void);
+SS_API int32_t ss_timing_count(void);
+SS_API ss_status ss_timing_query(int32_t i, char* name, int32_t name_len, int32_t* launches,
+                          double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAMPLED_CE_H */

@@ -1,0 +1,505 @@
+// ce_kernels.cu -- the memory- and latency-bound steps of the sampled-softmax
+// CE head: candidate build, row gather, LSE combine / loss reduction, dlogits
+// and the zero rows of the dense lm_head gradient.
+#include <limits.h>
+
+#include "sm100.cuh"
+#include "ss_internal.h"
+
+namespace ssb {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+constexpr int kBuildThreads = 1024;
+
+// ----------------------------------------------------------------------------
+// Candidate build (sampled_softmax.py, CandidateBuilder.build / _negatives)
+// ----------------------------------------------------------------------------
+
+// Exclusive prefix sum over the block; *total receives the block sum.
+__device__ int block_exclusive_scan(int x, int* total, int* s_warp) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nwarps = (blockDim.x + 31) >> 5;
+  int inc = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) s_warp[wid] = inc;
+  __syncthreads();
+  if (wid == 0) {
+    int w = lane < nwarps ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  const int before = wid > 0 ? s_warp[wid - 1] : 0;
+  *total = s_warp[nwarps - 1];
+  __syncthreads();
+  return before + inc - x;
+}
+
+__device__ __forceinline__ void write_status(int32_t* st, int code, int D, int need, int fallback,
+                                             int draw, int next_off, int bad, int marked) {
+  st[0] = code;
+  st[1] = D;
+  st[2] = need;
+  st[3] = fallback;
+  st[4] = draw;
+  st[5] = next_off;
+  st[6] = bad;
+  st[7] = marked;
+  for (int i = 8; i < SS_DEV_STATUS_WORDS; ++i) st[i] = 0;
+}
+
+// One CTA: target bitmap in shared memory, D, negative window or fallback,
+// then the bitmap and its per-word exclusive popcount prefix go to global.
+__global__ void __launch_bounds__(kBuildThreads)
+    k_build_mark(const int32_t* __restrict__ targets, int64_t T, int32_t V, int32_t P,
+                 int64_t offset, int32_t stride, uint32_t* __restrict__ g_bitmap,
+                 int32_t* __restrict__ g_prefix, int32_t* __restrict__ st) {
+  extern __shared__ uint32_t bm[];
+  __shared__ int s_warp[32];
+  __shared__ int s_bad;
+  const int tid = threadIdx.x;
+  const int NW = (V + 31) >> 5;
+
+  for (int w = tid; w < NW; w += kBuildThreads) bm[w] = 0u;
+  if (tid == 0) s_bad = INT_MAX;
+  __syncthreads();
+
+  // 1. mark every valid target (-1 = ignored; anything else outside [0, V) is an error)
+  {
+    const int64_t n4 = T >> 2;
+    const int4* t4 = reinterpret_cast<const int4*>(targets);
+    for (int64_t i = tid; i < n4; i += kBuildThreads) {
+      const int4 q = __ldg(t4 + i);
+      const int tv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = tv[j];
+        if (t == -1) continue;
+        if (t < -1 || t >= V) {
+          atomicMin(&s_bad, (int)min64(4 * i + j, INT_MAX));
+          continue;
+        }
+        atomicOr(&bm[t >> 5], 1u << (t & 31));
+      }
+    }
+    for (int64_t i = 4 * n4 + tid; i < T; i += kBuildThreads) {
+      const int t = __ldg(targets + i);
+      if (t == -1) continue;
+      if (t < -1 || t >= V) {
+        atomicMin(&s_bad, (int)min64(i, INT_MAX));
+        continue;
+      }
+      atomicOr(&bm[t >> 5], 1u << (t & 31));
+    }
+  }
+  __syncthreads();
+  if (s_bad != INT_MAX) {
+    if (tid == 0) write_status(st, SS_ERR_BAD_TARGET, 0, 0, 0, 0, (int)offset, s_bad, 0);
+    return;
+  }
+
+  // Each thread owns a contiguous run of bitmap words.
+  const int wper = (NW + kBuildThreads - 1) / kBuildThreads;
+  const int w_lo = min(NW, tid * wper), w_hi = min(NW, w_lo + wper);
+  const uint32_t last_mask = (V & 31) ? ((1u << (V & 31)) - 1u) : 0xffffffffu;
+
+  // 2. D = number of distinct valid targets
+  int local = 0;
+  for (int w = w_lo; w < w_hi; ++w) local += __popc(bm[w]);
+  int D;
+  block_exclusive_scan(local, &D, s_warp);
+  if (D > P) {
+    if (tid == 0) write_status(st, SS_ERR_TOO_MANY_TARGETS, D, 0, 0, 0, (int)offset, -1, D);
+    return;
+  }
+  const int need = P - D;
+  int draw = 0, fallback = 0;
+
+  if (need > 0) {
+    // 3. window of the stride sweep: positions offset .. offset+draw-1 (mod V)
+    draw = (int)min64((int64_t)V, (17LL * need) / 10 + 256);
+    const int kper = (draw + kBuildThreads - 1) / kBuildThreads;
+    const int k_lo = min(draw, tid * kper), k_hi = min(draw, k_lo + kper);
+    const int64_t smod = (int64_t)stride % V;
+    int64_t k0 = offset + k_lo;
+    if (k0 >= V) k0 -= V;
+    const int cls0 = (int)(((int64_t)stride % V) * k0 % V);
+
+    int cnt = 0;
+    {
+      int c = cls0;
+      for (int k = k_lo; k < k_hi; ++k) {
+        cnt += ((bm[c >> 5] >> (c & 31)) & 1u) ? 0 : 1;
+        c += (int)smod;
+        if (c >= V) c -= V;
+      }
+    }
+    int total;
+    const int base = block_exclusive_scan(cnt, &total, s_warp);
+    if (total >= need) {
+      // first `need` unmarked classes in sweep order. Classes in the window
+      // are distinct, so marking one never changes another's test.
+      int c = cls0, r = base;
+      for (int k = k_lo; k < k_hi && r < need; ++k) {
+        if (!((bm[c >> 5] >> (c & 31)) & 1u)) {
+          atomicOr(&bm[c >> 5], 1u << (c & 31));
+          ++r;
+        }
+        c += (int)smod;
+        if (c >= V) c -= V;
+      }
+    } else {
+      // fallback: evenly strided pick over the ascending unmarked classes
+      fallback = 1;
+      const int F = V - D;
+      if (F < need) {
+        if (tid == 0) write_status(st, SS_ERR_NO_FREE_CLASSES, D, need, 1, draw, (int)offset, -1, D);
+        return;
+      }
+      const int step = max(1, F / need);
+      int fcnt = 0;
+      for (int w = w_lo; w < w_hi; ++w)
+        fcnt += __popc(~bm[w] & (w == NW - 1 ? last_mask : 0xffffffffu));
+      int ftotal;
+      int r = block_exclusive_scan(fcnt, &ftotal, s_warp);
+      for (int w = w_lo; w < w_hi; ++w) {
+        uint32_t freeb = ~bm[w] & (w == NW - 1 ? last_mask : 0xffffffffu);
+        uint32_t pick = 0u;
+        while (freeb) {
+          const int b = __ffs(freeb) - 1;
+          freeb &= freeb - 1u;
+          if (r % step == 0 && r / step < need) pick |= 1u << b;
+          ++r;
+        }
+        bm[w] |= pick;
+      }
+    }
+  }
+  __syncthreads();
+
+  // 4. per-word exclusive prefix of the final marks -> global
+  int cnt = 0;
+  for (int w = w_lo; w < w_hi; ++w) cnt += __popc(bm[w]);
+  int marked;
+  int run = block_exclusive_scan(cnt, &marked, s_warp);
+  for (int w = w_lo; w < w_hi; ++w) {
+    const uint32_t b = bm[w];
+    g_bitmap[w] = b;
+    g_prefix[w] = run;
+    run += __popc(b);
+  }
+  if (tid == 0) {
+    const int next_off = (int)((offset + draw) % V);
+    write_status(st, marked == P ? SS_OK : SS_ERR_NO_FREE_CLASSES, D, need, fallback, draw,
+                 next_off, -1, marked);
+  }
+}
+
+// candidates / vocab_pos from the bitmap (threads [0, V)), target_pos (threads [V, V+T)).
+__global__ void k_build_emit(const int32_t* __restrict__ targets, int64_t T, int32_t V, int32_t P,
+                             const uint32_t* __restrict__ bitmap, const int32_t* __restrict__ prefix,
+                             const int32_t* __restrict__ st, int32_t* __restrict__ candidates,
+                             int32_t* __restrict__ target_pos, int32_t* __restrict__ vocab_pos) {
+  const int code = *reinterpret_cast<const volatile int32_t*>(st);
+  const int64_t n = (int64_t)V + T;
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    if (g < V) {
+      const int c = (int)g;
+      if (code != SS_OK) {
+        vocab_pos[c] = -1;
+        if (c < P) candidates[c] = -1;
+        continue;
+      }
+      const uint32_t bits = bitmap[c >> 5];
+      const int b = c & 31;
+      if ((bits >> b) & 1u) {
+        const int pos = prefix[c >> 5] + __popc(bits & ((1u << b) - 1u));
+        vocab_pos[c] = pos;
+        candidates[pos] = c;
+      } else {
+        vocab_pos[c] = -1;
+      }
+    } else {
+      const int64_t i = g - V;
+      const int t = __ldg(targets + i);
+      if (code != SS_OK || t < 0 || t >= V) {
+        target_pos[i] = -1;
+        continue;
+      }
+      const uint32_t bits = bitmap[t >> 5];
+      const int b = t & 31;
+      target_pos[i] = prefix[t >> 5] + __popc(bits & ((1u << b) - 1u));
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Row gather W_C[j] = lm_head[C_j] (sampled_softmax.py, _gather_rows): one warp
+// per row, 16-byte vectors.
+// ----------------------------------------------------------------------------
+__global__ void k_gather(const uint4* __restrict__ lm, const int32_t* __restrict__ cand, int32_t P,
+                         int32_t vec_per_row, int32_t V, uint4* __restrict__ w_c,
+                         int32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < P; r += warps) {
+    const int c = __ldg(cand + r);
+    uint4* dst = w_c + r * vec_per_row;
+    if (c < 0 || c >= V) {
+      for (int v = lane; v < vec_per_row; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+      if (lane == 0 && atomicCAS(status, 0, (int32_t)SS_ERR_BAD_INDEX) == 0) status[1] = 1;
+      continue;
+    }
+    const uint4* src = lm + (int64_t)c * vec_per_row;
+    int v = lane;
+    for (; v + 64 < vec_per_row; v += 96) {
+      const uint4 a = __ldg(src + v), b = __ldg(src + v + 32), d = __ldg(src + v + 64);
+      dst[v] = a;
+      dst[v + 32] = b;
+      dst[v + 64] = d;
+    }
+    for (; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// LSE combine: merge the per-tile (max, sum) pairs of each row; per-row loss;
+// per-block partial sums in a fixed order (deterministic).
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(kCombineThreads)
+    k_combine(const float2* __restrict__ stats, const float* __restrict__ zt,
+              const int32_t* __restrict__ tpos, int64_t T, int32_t P, int32_t tiles_n,
+              float* __restrict__ lse, double* __restrict__ partials) {
+  __shared__ double s_sum[kCombineThreads / 32];
+  __shared__ int s_cnt[kCombineThreads / 32];
+  const int64_t i = (int64_t)blockIdx.x * kCombineThreads + threadIdx.x;
+  double my = 0.0;
+  int cnt = 0;
+  if (i < T) {
+    float M = -INFINITY, S = 0.f;
+    for (int n = 0; n < tiles_n; ++n) {
+      const float2 p = stats[(int64_t)n * T + i];
+      if (p.x > M) {
+        S = S * ex2_approx((M - p.x) * kLog2e) + p.y;
+        M = p.x;
+      } else {
+        S += p.y * ex2_approx((p.x - M) * kLog2e);
+      }
+    }
+    const float l = M + logf(S);
+    lse[i] = l;
+    const int t = tpos[i];
+    if (t >= 0 && t < P) {
+      my = (double)l - (double)zt[i];
+      cnt = 1;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    my += __shfl_down_sync(0xffffffffu, my, o);
+    cnt += __shfl_down_sync(0xffffffffu, cnt, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    s_sum[threadIdx.x >> 5] = my;
+    s_cnt[threadIdx.x >> 5] = cnt;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    int c = 0;
+    for (int w = 0; w < kCombineThreads / 32; ++w) {
+      s += s_sum[w];
+      c += s_cnt[w];
+    }
+    partials[2 * blockIdx.x] = s;
+    partials[2 * blockIdx.x + 1] = (double)c;
+  }
+}
+
+__global__ void k_finalize(const double* __restrict__ partials, int32_t nblocks,
+                           float* __restrict__ loss, int32_t* __restrict__ n_valid) {
+  __shared__ double s_sum[32], s_cnt[32];
+  double s = 0.0, c = 0.0;
+  for (int b = threadIdx.x; b < nblocks; b += blockDim.x) {
+    s += partials[2 * b];
+    c += partials[2 * b + 1];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_down_sync(0xffffffffu, s, o);
+    c += __shfl_down_sync(0xffffffffu, c, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    s_sum[threadIdx.x >> 5] = s;
+    s_cnt[threadIdx.x >> 5] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double ts = 0.0, tc = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+      ts += s_sum[w];
+      tc += s_cnt[w];
+    }
+    *n_valid = (int32_t)tc;
+    *loss = tc > 0.0 ? (float)(ts / tc) : 0.f;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// dlogits in place: G = (g / n) (exp(z - lse) - onehot), 0 on ignored rows
+// ("Learning Triton ... Softmax", section "Gradient").
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__global__ void __launch_bounds__(256)
+    k_dlogits(uint16_t* __restrict__ z, int64_t T, int32_t P, int64_t ldz,
+              const float* __restrict__ lse, const int32_t* __restrict__ tpos,
+              const float* __restrict__ grad_loss, const int32_t* __restrict__ n_valid) {
+  const int nv = *n_valid;
+  const float coef = nv > 0 ? *grad_loss / (float)nv : 0.f;
+  const int vpr = (int)(ldz >> 3);  // 16-byte vectors per row
+  for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
+    uint4* zr = reinterpret_cast<uint4*>(z + row * ldz);
+    const int t = __ldg(tpos + row);
+    if (t < 0 || t >= P || coef == 0.f) {
+      for (int v = threadIdx.x; v < vpr; v += blockDim.x) __stcs(zr + v, make_uint4(0, 0, 0, 0));
+      continue;
+    }
+    const float l2 = __ldg(lse + row) * kLog2e;
+    for (int v0 = threadIdx.x; v0 < vpr; v0 += 4 * blockDim.x) {
+      uint4 in[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * blockDim.x;
+        if (v < vpr) in[u] = __ldcs(zr + v);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * blockDim.x;
+        if (v < vpr) {
+          const uint32_t w[4] = {in[u].x, in[u].y, in[u].z, in[u].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int c = v * 8 + 2 * h;
+            float a = coef * ex2_approx(fmaf(bf16_lo(w[h]), kLog2e, -l2));
+            float b = coef * ex2_approx(fmaf(bf16_hi(w[h]), kLog2e, -l2));
+            if (c == t) a -= coef;
+            if (c + 1 == t) b -= coef;
+            if (c >= P) a = 0.f;
+            if (c + 1 >= P) b = 0.f;
+            o[h] = pack_bf16x2(a, b);
+          }
+          __stcs(zr + v, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+      }
+    }
+  }
+}
+
+// dW rows outside C (or every row) set to +0.0.
+__global__ void k_zero_rows(uint4* __restrict__ dW, int32_t V, int32_t vec_per_row,
+                            const int32_t* __restrict__ vocab_pos, int all_rows) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < V; r += warps) {
+    if (!all_rows && __ldg(vocab_pos + r) >= 0) continue;
+    uint4* dst = dW + r * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) __stcs(dst + v, make_uint4(0, 0, 0, 0));
+  }
+}
+
+// ----------------------------------------------------------------------------
+// launchers
+// ----------------------------------------------------------------------------
+static int g_sms_cache = 0;
+static int num_sms() {
+  if (g_sms_cache == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_sms_cache, cudaDevAttrMultiProcessorCount, dev);
+    if (g_sms_cache <= 0) g_sms_cache = 148;
+  }
+  return g_sms_cache;
+}
+
+cudaError_t launch_build_mark(const int32_t* targets, int64_t T, int32_t V, int32_t P,
+                              int64_t offset, int32_t stride, uint32_t* bitmap, int32_t* prefix,
+                              int32_t* dev_status, cudaStream_t s) {
+  const int smem = ((V + 31) / 32) * 4;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_build_mark, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (SS_MAX_VOCAB / 32) * 4);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_build_mark<<<1, kBuildThreads, smem, s>>>(targets, T, V, P, offset, stride, bitmap, prefix,
+                                              dev_status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_emit(const int32_t* targets, int64_t T, int32_t V, int32_t P,
+                              const uint32_t* bitmap, const int32_t* prefix,
+                              const int32_t* dev_status, int32_t* candidates,
+                              int32_t* target_pos, int32_t* vocab_pos, cudaStream_t s) {
+  const int64_t n = (int64_t)V + T;
+  const int blocks = (int)min64((n + 255) / 256, (int64_t)num_sms() * 8);
+  k_build_emit<<<blocks, 256, 0, s>>>(targets, T, V, P, bitmap, prefix, dev_status, candidates,
+                                      target_pos, vocab_pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const uint16_t* lm_head, const int32_t* cand, int32_t P, int32_t d,
+                          int32_t V, uint16_t* w_c, int32_t* status, cudaStream_t s) {
+  const int warps_per_block = 8;
+  const int blocks = (int)min64((P + warps_per_block - 1) / warps_per_block,
+                                       (int64_t)num_sms() * 16);
+  k_gather<<<blocks, warps_per_block * 32, 0, s>>>(reinterpret_cast<const uint4*>(lm_head), cand, P,
+                                                    d / 8, V, reinterpret_cast<uint4*>(w_c), status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float2* stats, const float* zt, const int32_t* tpos, int64_t T,
+                           int32_t P, int32_t tiles_n, float* lse, double* partials,
+                           int32_t nblocks, cudaStream_t s) {
+  if (nblocks == 0) return cudaSuccess;
+  k_combine<<<nblocks, kCombineThreads, 0, s>>>(stats, zt, tpos, T, P, tiles_n, lse, partials);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const double* partials, int32_t nblocks, float* loss,
+                            int32_t* n_valid, cudaStream_t s) {
+  k_finalize<<<1, 1024, 0, s>>>(partials, nblocks, loss, n_valid);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dlogits(uint16_t* z, int64_t T, int32_t P, int64_t ldz, const float* lse,
+                           const int32_t* tpos, const float* grad_loss, const int32_t* n_valid,
+                           cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = (int)min64(T, (int64_t)num_sms() * 8);
+  k_dlogits<<<blocks, 256, 0, s>>>(z, T, P, ldz, lse, tpos, grad_loss, n_valid);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_rows(uint16_t* dW, int32_t V, int32_t d, const int32_t* vocab_pos,
+                             int all_rows, cudaStream_t s) {
+  const int blocks = (int)min64((V + 7) / 8, (int64_t)num_sms() * 16);
+  k_zero_rows<<<blocks, 256, 0, s>>>(reinterpret_cast<uint4*>(dW), V, d / 8, vocab_pos, all_rows);
+  return cudaGetLastError();
+}
+
+}  // namespace ssb

@@ -1,0 +1,418 @@
+// ss_api.cu -- the C ABI declared in include/sampled_ce.h: argument checks,
+// workspace layout, TMA descriptors and the launch sequence of each call.
+#include <cudaTypedefs.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "ss_internal.h"
+
+using namespace ssb;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+ss_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
+  return SS_ERR_CUDA;
+}
+
+#define SS_CUDA(call, where)                        \
+  do {                                              \
+    cudaError_t _e = (call);                        \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+// ------------------------------------------------------------- device info --
+struct DeviceState {
+  bool ready = false;
+  int sms = 0;
+  ss_status status = SS_OK;
+};
+std::mutex g_dev_mu;
+DeviceState g_dev[128];
+
+ss_status ensure_device(int* sms) {
+  int dev = 0;
+  SS_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 128) return SS_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0;
+    SS_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev),
+            "cudaDeviceGetAttribute");
+    SS_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev),
+            "cudaDeviceGetAttribute");
+    if (major != 10) {
+      d.status = SS_ERR_UNSUPPORTED_DEVICE;
+    } else {
+      for (int k = 0; k < 3; ++k)
+        SS_CUDA(cudaFuncSetAttribute(gemm_kernel_ptr(k),
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     gemm_smem_bytes()),
+                "cudaFuncSetAttribute");
+    }
+    d.ready = true;
+  }
+  *sms = d.sms;
+  return d.status;
+}
+
+// --------------------------------------------------------------- TMA maps --
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [outer][inner] with row pitch `row_elems`, 128-byte swizzle.
+ss_status make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
+                   uint64_t row_elems, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+    return SS_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_elems * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SS_ERR_CUDA;
+  }
+  return SS_OK;
+}
+
+// ----------------------------------------------------------------- timing --
+struct TimingState {
+  bool on = false;
+  std::vector<cudaEvent_t> ev;        // pairs
+  std::vector<int> rec_name;          // name index per used pair
+  std::vector<std::string> names;
+  size_t used = 0;
+};
+TimingState g_tm;
+constexpr size_t kTimingPairs = 8192;
+
+int timing_begin(const char* name, cudaStream_t s) {
+  if (!g_tm.on || g_tm.used >= kTimingPairs) return -1;
+  if (g_tm.ev.empty()) {
+    g_tm.ev.resize(2 * kTimingPairs);
+    for (auto& e : g_tm.ev) cudaEventCreate(&e);
+  }
+  int idx = -1;
+  for (size_t i = 0; i < g_tm.names.size(); ++i)
+    if (g_tm.names[i] == name) idx = (int)i;
+  if (idx < 0) {
+    g_tm.names.push_back(name);
+    idx = (int)g_tm.names.size() - 1;
+  }
+  const size_t slot = g_tm.used++;
+  g_tm.rec_name.push_back(idx);
+  cudaEventRecord(g_tm.ev[2 * slot], s);
+  return (int)slot;
+}
+
+void timing_end(int slot, cudaStream_t s) {
+  if (slot >= 0) cudaEventRecord(g_tm.ev[2 * slot + 1], s);
+}
+
+#define SS_LAUNCH(name, stream, call)                         \
+  do {                                                        \
+    const int _slot = timing_begin(name, stream);             \
+    cudaError_t _e = (call);                                  \
+    timing_end(_slot, stream);                                \
+    if (_e != cudaSuccess) return cuda_fail(_e, name);        \
+  } while (0)
+
+// -------------------------------------------------------------- workspace --
+constexpr int kBM = 128, kBN = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Layout {
+  size_t bitmap, prefix, partials, w_c, z, stats, zt, total;
+  int64_t ldz;
+  int tiles_n;
+  int nblk;
+};
+
+bool sizes_ok(int64_t T, int32_t d, int32_t V, int32_t P) {
+  return T >= 0 && T <= INT32_MAX && d >= 8 && d % 8 == 0 && d <= (1 << 16) && V >= 1 &&
+         V <= SS_MAX_VOCAB && P >= 1 && P <= V;
+}
+
+Layout layout(int64_t T, int32_t d, int32_t V, int32_t P) {
+  Layout L;
+  const size_t nw = (size_t)(V + 31) / 32;
+  L.ldz = (P + 7) / 8 * 8;
+  L.tiles_n = (P + kBN - 1) / kBN;
+  L.nblk = combine_blocks(T);
+  size_t off = 0;
+  L.bitmap = off;
+  off += align_up(nw * 4, 256);
+  L.prefix = off;
+  off += align_up(nw * 4, 256);
+  L.partials = off;
+  off += align_up((size_t)L.nblk * 16 + 16, 256);
+  off = align_up(off, 1024);
+  L.w_c = off;
+  off += align_up((size_t)P * d * 2, 1024);
+  L.z = off;
+  off += align_up((size_t)T * L.ldz * 2, 1024);
+  L.stats = off;
+  off += align_up((size_t)L.tiles_n * T * 8, 256);
+  L.zt = off;
+  off += align_up((size_t)T * 4, 256);
+  L.total = off;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int gcd_int(int64_t a, int64_t b) {
+  while (b) {
+    const int64_t t = a % b;
+    a = b;
+    b = t;
+  }
+  return (int)a;
+}
+
+}  // namespace
+
+// ===================================================================== API ==
+extern "C" {
+
+int32_t ss_version(void) { return 10000; }
+
+const char* ss_last_cuda_error(void) { return g_last_error; }
+
+const char* ss_status_string(int32_t s) {
+  switch (s) {
+    case SS_OK: return "ok";
+    case SS_ERR_INVALID_ARG: return "invalid argument";
+    case SS_ERR_BAD_TARGET: return "target outside [-1, V)";
+    case SS_ERR_TOO_MANY_TARGETS: return "more distinct targets than candidates (D > P)";
+    case SS_ERR_NO_FREE_CLASSES: return "not enough free classes for the negatives";
+    case SS_ERR_STRIDE_NOT_COPRIME: return "stride not coprime with V";
+    case SS_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case SS_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case SS_ERR_CUDA: return "CUDA runtime error";
+    case SS_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100 (B200)";
+    case SS_ERR_KERNEL_TIMEOUT: return "kernel pipeline wait timed out";
+    case SS_ERR_BAD_INDEX: return "candidate or position index out of range";
+    default: return "unknown status";
+  }
+}
+
+size_t ss_workspace_bytes(int64_t T, int32_t d, int32_t V, int32_t P) {
+  if (!sizes_ok(T, d, V, P)) return 0;
+  return layout(T, d, V, P).total;
+}
+
+size_t ss_build_workspace_bytes(int32_t V) {
+  if (V < 1 || V > SS_MAX_VOCAB) return 0;
+  return 2 * align_up((size_t)(V + 31) / 32 * 4, 256);
+}
+
+ss_status ss_build_candidates(const int32_t* targets, int64_t T, int32_t V, int32_t P,
+                              int64_t offset, int32_t stride, int32_t* candidates,
+                              int32_t* target_pos, int32_t* vocab_pos, int32_t* dev_status,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 0 || T > INT32_MAX || V < 1 || V > SS_MAX_VOCAB || P < 1 || P > V || offset < 0 ||
+      stride < 1)
+    return SS_ERR_INVALID_ARG;
+  if (gcd_int(stride, V) != 1) return SS_ERR_STRIDE_NOT_COPRIME;
+  if ((T > 0 && targets == nullptr) || candidates == nullptr || vocab_pos == nullptr ||
+      (T > 0 && target_pos == nullptr) || dev_status == nullptr || workspace == nullptr)
+    return SS_ERR_INVALID_ARG;
+  if ((T > 0 && !aligned16(targets)) || !aligned16(workspace)) return SS_ERR_MISALIGNED;
+  const size_t nw = (size_t)(V + 31) / 32;
+  if (workspace_bytes < ss_build_workspace_bytes(V)) return SS_ERR_WORKSPACE_TOO_SMALL;
+  int sms;
+  ss_status ds = ensure_device(&sms);
+  if (ds != SS_OK) return ds;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(ws);
+  int32_t* prefix = reinterpret_cast<int32_t*>(ws + align_up(nw * 4, 256));
+  SS_LAUNCH("build_mark", s,
+            launch_build_mark(targets, T, V, P, offset % V, stride, bitmap, prefix, dev_status, s));
+  SS_LAUNCH("build_emit", s,
+            launch_build_emit(targets, T, V, P, bitmap, prefix, dev_status, candidates, target_pos,
+                              vocab_pos, s));
+  return SS_OK;
+}
+
+ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t* candidates,
+                        const int32_t* target_pos, int64_t T, int32_t d, int32_t V, int32_t P,
+                        float* loss, float* lse, int32_t* n_valid, int32_t* dev_status,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (!sizes_ok(T, d, V, P)) return SS_ERR_INVALID_ARG;
+  if (lm_head == nullptr || candidates == nullptr || loss == nullptr || n_valid == nullptr ||
+      dev_status == nullptr || workspace == nullptr ||
+      (T > 0 && (x == nullptr || target_pos == nullptr || lse == nullptr)))
+    return SS_ERR_INVALID_ARG;
+  if (!aligned16(lm_head) || !aligned16(workspace) || (T > 0 && !aligned16(x)))
+    return SS_ERR_MISALIGNED;
+  const Layout L = layout(T, d, V, P);
+  if (workspace_bytes < L.total) return SS_ERR_WORKSPACE_TOO_SMALL;
+  int sms;
+  ss_status ds = ensure_device(&sms);
+  if (ds != SS_OK) return ds;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* w_c = reinterpret_cast<uint16_t*>(ws + L.w_c);
+  uint16_t* z = reinterpret_cast<uint16_t*>(ws + L.z);
+  float2* stats = reinterpret_cast<float2*>(ws + L.stats);
+  float* zt = reinterpret_cast<float*>(ws + L.zt);
+  double* partials = reinterpret_cast<double*>(ws + L.partials);
+  int32_t* kstatus = dev_status + 8;
+
+  SS_LAUNCH("gather", s, launch_gather(lm_head, candidates, P, d, V, w_c, kstatus, s));
+  if (T > 0) {
+    CUtensorMap ta, tb, tc;
+    ss_status r;
+    if ((r = make_map(&ta, x, d, T, d, 64, kBM)) != SS_OK) return r;
+    if ((r = make_map(&tb, w_c, d, P, d, 64, kBN)) != SS_OK) return r;
+    if ((r = make_map(&tc, z, P, T, L.ldz, 64, 32)) != SS_OK) return r;
+    GemmArgs a{};
+    a.M = (int32_t)T;
+    a.N = P;
+    a.K = d;
+    a.tiles_m = (int32_t)((T + kBM - 1) / kBM);
+    a.tiles_n = L.tiles_n;
+    a.num_kb = (d + 63) / 64;
+    a.tpos = target_pos;
+    a.stats = stats;
+    a.zt = zt;
+    a.status = kstatus;
+    const int tiles = a.tiles_m * a.tiles_n;
+    SS_LAUNCH("fwd_gemm_ce", s, launch_gemm(KIND_FWD, ta, tb, tc, a, tiles < sms ? tiles : sms, s));
+    SS_LAUNCH("lse_combine", s,
+              launch_combine(stats, zt, target_pos, T, P, L.tiles_n, lse, partials, L.nblk, s));
+  }
+  SS_LAUNCH("loss_finalize", s, launch_finalize(partials, L.nblk, loss, n_valid, s));
+  return SS_OK;
+}
+
+ss_status ss_ce_backward(const float* grad_loss, const ss_bf16* x, const int32_t* candidates,
+                         const int32_t* target_pos, const int32_t* vocab_pos, const float* lse,
+                         const int32_t* n_valid, int64_t T, int32_t d, int32_t V, int32_t P,
+                         ss_bf16* dx, ss_bf16* dW, int32_t* dev_status, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (!sizes_ok(T, d, V, P)) return SS_ERR_INVALID_ARG;
+  if (grad_loss == nullptr || candidates == nullptr || vocab_pos == nullptr ||
+      n_valid == nullptr || dW == nullptr || dev_status == nullptr || workspace == nullptr ||
+      (T > 0 && (x == nullptr || target_pos == nullptr || lse == nullptr || dx == nullptr)))
+    return SS_ERR_INVALID_ARG;
+  if (!aligned16(dW) || !aligned16(workspace) || (T > 0 && (!aligned16(x) || !aligned16(dx))))
+    return SS_ERR_MISALIGNED;
+  const Layout L = layout(T, d, V, P);
+  if (workspace_bytes < L.total) return SS_ERR_WORKSPACE_TOO_SMALL;
+  int sms;
+  ss_status ds = ensure_device(&sms);
+  if (ds != SS_OK) return ds;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* w_c = reinterpret_cast<uint16_t*>(ws + L.w_c);
+  uint16_t* z = reinterpret_cast<uint16_t*>(ws + L.z);
+  int32_t* kstatus = dev_status + 8;
+
+  if (T == 0) {
+    SS_LAUNCH("zero_rows", s, launch_zero_rows(dW, V, d, vocab_pos, 1, s));
+    return SS_OK;
+  }
+  SS_LAUNCH("dlogits", s, launch_dlogits(z, T, P, L.ldz, lse, target_pos, grad_loss, n_valid, s));
+  SS_LAUNCH("zero_rows", s, launch_zero_rows(dW, V, d, vocab_pos, 0, s));
+
+  CUtensorMap ga, wb, dxs, ga2, xb;
+  ss_status r;
+  if ((r = make_map(&ga, z, P, T, L.ldz, 64, kBM)) != SS_OK) return r;   // G, K-major
+  if ((r = make_map(&wb, w_c, d, P, d, 64, 64)) != SS_OK) return r;      // W_C, MN-major
+  if ((r = make_map(&dxs, dx, d, T, d, 64, 32)) != SS_OK) return r;      // dx store
+  if ((r = make_map(&ga2, z, P, T, L.ldz, 64, 64)) != SS_OK) return r;   // G^T, MN-major
+  if ((r = make_map(&xb, x, d, T, d, 64, 64)) != SS_OK) return r;        // x, MN-major
+
+  GemmArgs a{};
+  a.M = (int32_t)T;
+  a.N = d;
+  a.K = P;
+  a.tiles_m = (int32_t)((T + kBM - 1) / kBM);
+  a.tiles_n = (d + kBN - 1) / kBN;
+  a.num_kb = (P + 63) / 64;
+  a.status = kstatus;
+  int tiles = a.tiles_m * a.tiles_n;
+  SS_LAUNCH("dx_gemm", s, launch_gemm(KIND_DX, ga, wb, dxs, a, tiles < sms ? tiles : sms, s));
+
+  GemmArgs b{};
+  b.M = P;
+  b.N = d;
+  b.K = (int32_t)T;
+  b.tiles_m = (P + kBM - 1) / kBM;
+  b.tiles_n = (d + kBN - 1) / kBN;
+  b.num_kb = (int32_t)((T + 63) / 64);
+  b.cand = candidates;
+  b.dW = dW;
+  b.V = V;
+  b.status = kstatus;
+  tiles = b.tiles_m * b.tiles_n;
+  SS_LAUNCH("dw_gemm_scatter", s, launch_gemm(KIND_DW, ga2, xb, ga2, b, tiles < sms ? tiles : sms, s));
+  return SS_OK;
+}
+
+ss_status ss_timing_enable(int32_t enable) {
+  g_tm.on = enable != 0;
+  return SS_OK;
+}
+
+ss_status ss_timing_reset(void) {
+  g_tm.used = 0;
+  g_tm.rec_name.clear();
+  g_tm.names.clear();
+  return SS_OK;
+}
+
+int32_t ss_timing_count(void) { return (int32_t)g_tm.names.size(); }
+
+ss_status ss_timing_query(int32_t i, char* name, int32_t name_len, int32_t* launches,
+                          double* total_ms) {
+  if (i < 0 || i >= (int32_t)g_tm.names.size()) return SS_ERR_INVALID_ARG;
+  if (name != nullptr && name_len > 0) {
+    strncpy(name, g_tm.names[i].c_str(), (size_t)name_len - 1);
+    name[name_len - 1] = '\0';
+  }
+  int n = 0;
+  double tot = 0.0;
+  for (size_t k = 0; k < g_tm.used; ++k) {
+    if (g_tm.rec_name[k] != i) continue;
+    SS_CUDA(cudaEventSynchronize(g_tm.ev[2 * k + 1]), "cudaEventSynchronize");
+    float ms = 0.f;
+    SS_CUDA(cudaEventElapsedTime(&ms, g_tm.ev[2 * k], g_tm.ev[2 * k + 1]), "cudaEventElapsedTime");
+    tot += ms;
+    ++n;
+  }
+  if (launches) *launches = n;
+  if (total_ms) *total_ms = tot;
+  return SS_OK;
+}
+
+}  // extern "C"

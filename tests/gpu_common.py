@@ -1,0 +1,106 @@
+"""Shared helpers for the GPU parity tests (not collected by pytest).
+
+Runs the CUDA path through the C ABI (via the ctypes binding) and the float64
+oracle on the same seeded inputs, and holds the tolerances:
+
+* candidate set, target/vocab positions, builder info, dW zero pattern:
+  bit-exact;
+* loss: relative 1e-3; lse: absolute 1e-3 (both come from fp32 accumulators);
+* dX and dW (rows in C): relative Frobenius error 2e-2 (bf16 outputs from bf16
+  logits), with max-abs error / max |expected| reported.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import sampled_ce as oc
+from sampled_softmax_cross_b200 import capi
+from sampled_softmax_cross_b200 import workloads as wl
+
+LOSS_RTOL = 1e-3
+LSE_ATOL = 1e-3
+GRAD_RTOL = 2e-2
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def run_build(targets: np.ndarray, V: int, P: int, offset: int, stride: int = 20011):
+    T = targets.size
+    dev = torch.device("cuda")
+    ws = torch.empty(capi.ss_build_workspace_bytes(V), dtype=torch.uint8, device=dev)
+    cand = torch.empty(P, dtype=torch.int32, device=dev)
+    tpos = torch.empty(max(T, 1), dtype=torch.int32, device=dev)
+    vpos = torch.empty(V, dtype=torch.int32, device=dev)
+    st = torch.zeros(capi.DEV_STATUS_WORDS, dtype=torch.int32, device=dev)
+    t = torch.from_numpy(np.ascontiguousarray(targets, dtype=np.int32)).cuda()
+    capi.ss_build_candidates(t, V, P, offset, stride, cand, tpos, vpos, st, ws)
+    torch.cuda.synchronize()
+    return cand.cpu().numpy(), tpos[:T].cpu().numpy(), vpos.cpu().numpy(), st.tolist()
+
+
+def check_build(targets, V, P, offset, stride=20011):
+    cand, tpos, vpos, st = run_build(targets, V, P, offset, stride)
+    ocand, otpos, ovpos, info = oc.build_candidates(targets, V, P, offset, stride)
+    assert st[0] == 0, st
+    assert np.array_equal(cand, ocand)
+    assert np.array_equal(tpos, otpos)
+    assert np.array_equal(vpos, ovpos)
+    assert st[1:6] == [info["D"], info["need"], int(info["used_fallback"]), info["draw"],
+                       info["next_offset"]], (st, info)
+    assert st[7] == P
+    return info
+
+
+def run_path(x_bits, lm_bits, targets, P, offset, stride=20011, grad=1.0):
+    """build + forward + backward on the GPU; numpy results."""
+    T, d = x_bits.shape
+    V = lm_bits.shape[0]
+    ce = capi.SampledCE(T, d, V, P)
+    x = dev_bf16(x_bits) if T else torch.empty((1, d), dtype=torch.bfloat16, device="cuda")
+    lm = dev_bf16(lm_bits)
+    t = torch.from_numpy(np.ascontiguousarray(targets, dtype=np.int32)).cuda()
+    ce.grad_loss.fill_(grad)
+    ce.step(t, x, lm, offset, stride)
+    torch.cuda.synchronize()
+    return dict(
+        candidates=ce.candidates.cpu().numpy(), target_pos=ce.target_pos[:T].cpu().numpy(),
+        vocab_pos=ce.vocab_pos.cpu().numpy(), status=ce.status(), loss=float(ce.loss.item()),
+        n_valid=int(ce.n_valid.item()), lse=ce.lse[:T].cpu().numpy().astype(np.float64),
+        dx_bits=host_bits(ce.dx[:T]), dW_bits=host_bits(ce.dW))
+
+
+def rel_fro(got: np.ndarray, want: np.ndarray) -> float:
+    den = np.linalg.norm(want)
+    return float(np.linalg.norm(got - want) / den) if den > 0 else float(np.linalg.norm(got))
+
+
+def compare_full(g: dict, o: dict, targets: np.ndarray):
+    """Element-by-element comparison against a full oracle run."""
+    assert g["status"][0] == 0 and g["status"][8] == 0, g["status"]
+    assert np.array_equal(g["candidates"], o["candidates"])
+    assert np.array_equal(g["target_pos"], o["target_pos"])
+    assert np.array_equal(g["vocab_pos"], o["vocab_pos"])
+    assert g["n_valid"] == o["n_valid"]
+    if o["n_valid"]:
+        assert abs(g["loss"] - o["loss"]) <= LOSS_RTOL * abs(o["loss"]), (g["loss"], o["loss"])
+    else:
+        assert g["loss"] == 0.0
+    if targets.size:
+        assert np.max(np.abs(g["lse"] - o["lse"])) <= LSE_ATOL
+    dx = wl.bits_to_f64(g["dx_bits"])
+    assert rel_fro(dx, o["dx"]) <= GRAD_RTOL, rel_fro(dx, o["dx"])
+    ign = o["target_pos"] < 0
+    assert np.all(g["dx_bits"][ign] == 0)
+    in_c = np.zeros(g["dW_bits"].shape[0], bool)
+    in_c[o["candidates"]] = True
+    assert np.all(g["dW_bits"][~in_c] == 0)  # +0.0 bits outside C
+    dW = wl.bits_to_f64(g["dW_bits"])
+    assert rel_fro(dW[in_c], o["dW"][in_c]) <= GRAD_RTOL, rel_fro(dW[in_c], o["dW"][in_c])

@@ -1,0 +1,122 @@
+"""C-ABI library: loads, exports every declared symbol, host-side checks.
+
+No kernel runs here: each call below is rejected by the host-side argument
+checks before any CUDA call, or is a pure host query.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from sampled_softmax_cross_b200 import build_lib, capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sampled_ce.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return capi.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ss_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("ss_build_candidates", "ss_ce_forward", "ss_ce_backward", "ss_workspace_bytes"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(capi.EXPORTS) == set(names)
+
+
+def test_status_strings(lib):
+    assert capi.ss_status_string(0) == "ok"
+    for code in range(1, 12):
+        assert capi.ss_status_string(code) != "unknown status"
+    assert capi.ss_status_string(999) == "unknown status"
+    assert capi.ss_version() >= 10000
+
+
+def test_workspace_bytes_rejects_bad_sizes(lib):
+    assert capi.ss_workspace_bytes(512, 128, 50304, 2048) > 0
+    assert capi.ss_workspace_bytes(512, 127, 50304, 2048) == 0   # d % 8
+    assert capi.ss_workspace_bytes(512, 128, 50304, 50305) == 0  # P > V
+    assert capi.ss_workspace_bytes(512, 128, 50304, 0) == 0
+    assert capi.ss_workspace_bytes(-1, 128, 50304, 2048) == 0
+    assert capi.ss_workspace_bytes(0, 128, 50304, 2048) > 0
+    assert capi.ss_workspace_bytes(512, 128, (1 << 19) + 1, 2048) == 0
+
+
+def test_workspace_holds_logits_and_rows(lib):
+    T, d, V, P = 49152, 768, 50304, 24576
+    ws = capi.ss_workspace_bytes(T, d, V, P)
+    assert ws >= T * P * 2 + P * d * 2 + T * 4
+    assert ws < T * P * 2 * 1.05
+    # padded logit rows when P is not a multiple of 8
+    assert capi.ss_workspace_bytes(100, 64, 5000, 1001) >= 100 * 1008 * 2
+
+
+def _raw(lib, fn, *args):
+    return getattr(lib, fn)(*args)
+
+
+@pytest.mark.parametrize("T,V,P,stride,offset,code", [
+    (10, 100, 0, 20011, 0, "SS_ERR_INVALID_ARG"),
+    (10, 100, 101, 20011, 0, "SS_ERR_INVALID_ARG"),
+    (10, 0, 1, 20011, 0, "SS_ERR_INVALID_ARG"),
+    (10, (1 << 19) + 1, 8, 20011, 0, "SS_ERR_INVALID_ARG"),
+    (10, 100, 10, 20011, -1, "SS_ERR_INVALID_ARG"),
+    (10, 100, 10, 0, 0, "SS_ERR_INVALID_ARG"),
+    (10, 100, 10, 10, 0, "SS_ERR_STRIDE_NOT_COPRIME"),
+    (10, 50304, 10, 3, 0, "SS_ERR_STRIDE_NOT_COPRIME"),
+])
+def test_build_host_rejections(lib, T, V, P, stride, offset, code):
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: rejected before any CUDA call
+    r = lib.ss_build_candidates(fake, T, V, P, offset, stride, fake, fake, fake, fake, fake,
+                                1 << 30, None)
+    assert r == capi.STATUS[code]
+
+
+def test_build_rejects_null_and_misaligned(lib):
+    a = ctypes.c_void_p(1 << 20)
+    r = lib.ss_build_candidates(None, 10, 100, 10, 0, 20011, a, a, a, a, a, 1 << 30, None)
+    assert r == capi.STATUS["SS_ERR_INVALID_ARG"]
+    mis = ctypes.c_void_p((1 << 20) + 4)
+    r = lib.ss_build_candidates(mis, 10, 100, 10, 0, 20011, a, a, a, a, a, 1 << 30, None)
+    assert r == capi.STATUS["SS_ERR_MISALIGNED"]
+    r = lib.ss_build_candidates(a, 10, 100, 10, 0, 20011, a, a, a, a, a, 16, None)
+    assert r == capi.STATUS["SS_ERR_WORKSPACE_TOO_SMALL"]
+
+
+def test_forward_backward_host_rejections(lib):
+    a = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    ws = capi.ss_workspace_bytes(512, 128, 50304, 2048)
+    f = lib.ss_ce_forward
+    assert f(a, a, a, a, 512, 100, 50304, 2048, a, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    assert f(a, a, a, a, 512, 128, 50304, 2048, a, a, a, a, a, ws - 1, None) == capi.STATUS["SS_ERR_WORKSPACE_TOO_SMALL"]
+    assert f(mis, a, a, a, 512, 128, 50304, 2048, a, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_MISALIGNED"]
+    assert f(a, None, a, a, 512, 128, 50304, 2048, a, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    b = lib.ss_ce_backward
+    assert b(a, a, a, a, a, a, a, 512, 128, 50304, 2049 * 0 + 50305, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    assert b(a, a, a, a, a, a, a, 512, 128, 50304, 2048, a, mis, a, a, ws, None) == capi.STATUS["SS_ERR_MISALIGNED"]
+    assert b(None, a, a, a, a, a, a, 512, 128, 50304, 2048, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(capi, "_lib", None)
+    with pytest.raises(capi.LibraryNotBuilt):
+        capi.load(str(tmp_path / "nope.so"))

@@ -1,0 +1,238 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle.
+
+Small and ragged shapes are compared element by element with a full oracle
+run. The five named workloads are run at full size in the launch
+configuration the benchmark times; their integer outputs are compared in full
+and their floating outputs on all rows (loss, lse) or on seeded samples of
+rows (dX) and of candidate columns (dW), which the oracle computes one by one.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sampled_ce as oc
+from sampled_softmax_cross_b200 import capi
+from sampled_softmax_cross_b200 import workloads as wl
+
+from gpu_common import (GRAD_RTOL, LOSS_RTOL, LSE_ATOL, check_build, compare_full, rel_fro,
+                        run_build, run_path)
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def oracle_run(x_bits, lm_bits, targets, P, offset, stride=20011, grad=1.0):
+    return oc.sampled_ce(wl.bits_to_f64(x_bits), wl.bits_to_f64(lm_bits), targets, P, offset,
+                         stride, grad_loss=grad)
+
+
+def random_case(T, d, V, P, seed, ignore_frac=0.05, zipf_s=1.1):
+    x, lm, t = wl.make_inputs(T, d, V, zipf_s, ignore_frac, seed)
+    D = np.unique(t[t >= 0]).size
+    assert D <= P
+    return x, lm, t
+
+
+# ----------------------------------------------------------- candidate build --
+
+@pytest.mark.parametrize("name", list(wl.WORKLOADS))
+def test_builder_bit_exact_on_workloads(name):
+    w = wl.WORKLOADS[name]
+    _, _, targets = wl.workload_inputs(w)
+    check_build(targets, w.V, w.P, w.offset)
+
+
+@pytest.mark.parametrize("case", json.load(open(os.path.join(GOLDEN, "builder_hand_worked.json")))["cases"],
+                         ids=lambda c: c["name"])
+def test_builder_hand_worked(case):
+    V = case["V"]
+    if "targets" in case:
+        t = np.array(case["targets"], np.int32)
+    else:
+        keep = [c for c in range(V) if c not in set(case["targets_all_except"])]
+        t = np.array(keep + [-1] * case["targets_extra_ignored"], np.int32)
+    info = check_build(t, V, case["P"], case["offset"], case["stride"])
+    assert info["used_fallback"] == case["used_fallback"]
+
+
+def test_builder_random_small_vocabularies():
+    rng = np.random.default_rng(11)
+    for V, stride in ((7, 3), (13, 5), (101, 20011), (263, 2), (1009, 20011), (5003, 20011)):
+        for _ in range(6):
+            T = int(rng.integers(0, 3 * V))
+            t = rng.integers(-1, V, T).astype(np.int32)
+            D = np.unique(t[t >= 0]).size
+            P = int(rng.integers(max(1, D), V + 1))
+            check_build(t, V, P, int(rng.integers(0, 4 * V)), stride)
+
+
+@pytest.mark.parametrize("V", [1009, 50304])
+def test_builder_forced_fallback(V):
+    rng = np.random.default_rng(V)
+    hits = 0
+    for _ in range(6):
+        off = int(rng.integers(V))
+        need = int(rng.integers(1, 40))
+        draw = min(V, (17 * need) // 10 + 256)
+        window = oc.stride_class(off + np.arange(draw), V)
+        keep_free = rng.choice(window, size=int(rng.integers(0, need)), replace=False)
+        t = np.setdiff1d(window, keep_free).astype(np.int32)
+        t = np.concatenate([t, rng.integers(0, V, 37).astype(np.int32), [-1, -1]]).astype(np.int32)
+        rng.shuffle(t)
+        D = np.unique(t[t >= 0]).size
+        info = check_build(t, V, min(V, D + need), off)
+        hits += info["used_fallback"]
+    assert hits >= 4
+
+
+def test_builder_edge_cases():
+    check_build(np.zeros(0, np.int32), 50304, 2048, 99)                      # empty microbatch
+    check_build(np.full(1000, -1, np.int32), 50304, 4096, 5)                  # all ignored
+    t = np.array([3, 17, 40, 3, -1], np.int32)
+    info = check_build(t, 101, 3, 7)                                          # D == P
+    assert info["draw"] == 0
+    check_build(np.array([0, 50303, 7], np.int32), 50304, 50304, 123)         # P == V
+    V = capi.MAX_VOCAB                                                        # largest vocabulary
+    rng = np.random.default_rng(3)
+    check_build(rng.integers(-1, V, 100000).astype(np.int32), V, 200000, 777, 20011)
+    check_build(rng.integers(0, 1000, 7).astype(np.int32), 1000, 999, 1, 7)   # T % 4 != 0
+
+
+def test_builder_device_errors():
+    _, _, _, st = run_build(np.array([1, 2, 3, 4], np.int32), 100, 3, 0)
+    assert st[0] == capi.STATUS["SS_ERR_TOO_MANY_TARGETS"] and st[1] == 4
+    cand, tpos, vpos, st = run_build(np.array([1, 2, 100, 5, -2], np.int32), 100, 10, 0)
+    assert st[0] == capi.STATUS["SS_ERR_BAD_TARGET"] and st[6] == 2
+    assert np.all(cand == -1) and np.all(tpos == -1) and np.all(vpos == -1)
+    with pytest.raises(capi.SampledCEError) as e:
+        run_build(np.array([1], np.int32), 50304, 8, 0, stride=6)
+    assert e.value.name == "SS_ERR_STRIDE_NOT_COPRIME"
+
+
+# ------------------------------------------------- full comparison, small --
+
+SMALL = [
+    # (T, d, V, P, seed, grad) -- several tiles and ragged tails in every dim
+    (512, 128, 50304, 2048, 0, 1.0),
+    (1000, 200, 5003, 3000, 1, 1.0),
+    (777, 136, 4099, 1001, 2, 2.5),
+    (300, 64, 1000, 1000, 3, 1.0),
+    (129, 8, 300, 257, 4, 0.5),
+    (2048, 768, 20023, 4096, 5, 1.0),
+]
+
+
+@pytest.mark.parametrize("T,d,V,P,seed,grad", SMALL)
+def test_small_shapes_match_oracle(T, d, V, P, seed, grad):
+    x, lm, t = random_case(T, d, V, P, seed)
+    off = (seed * 7919) % V
+    g = run_path(x, lm, t, P, off, grad=grad)
+    o = oracle_run(x, lm, t, P, off, grad=grad)
+    compare_full(g, o, t)
+
+
+def test_tiny_workload_matches_oracle():
+    w = wl.WORKLOADS["tiny"]
+    x, lm, t = wl.workload_inputs(w)
+    g = run_path(x, lm, t, w.P, w.offset)
+    o = oracle_run(x, lm, t, w.P, w.offset)
+    compare_full(g, o, t)
+
+
+def test_all_ignored_and_zero_grad():
+    x, lm, _ = random_case(256, 64, 2000, 512, 9)
+    t = np.full(256, -1, np.int32)
+    g = run_path(x, lm, t, 512, 3)
+    assert g["loss"] == 0.0 and g["n_valid"] == 0
+    assert np.all(g["dx_bits"] == 0) and np.all(g["dW_bits"] == 0)
+    x, lm, t = random_case(256, 64, 2000, 512, 10)
+    g = run_path(x, lm, t, 512, 3, grad=0.0)
+    assert np.all(wl.bits_to_f64(g["dx_bits"]) == 0) and np.all(wl.bits_to_f64(g["dW_bits"]) == 0)
+
+
+def test_empty_microbatch():
+    lm = wl.bf16_bits(np.random.default_rng(0).standard_normal((500, 64), dtype=np.float32))
+    g = run_path(np.zeros((0, 64), np.uint16), lm, np.zeros(0, np.int32), 100, 4)
+    assert g["loss"] == 0.0 and g["n_valid"] == 0
+    assert np.all(g["dW_bits"] == 0)
+
+
+def test_uniform_logits_give_log_p():
+    T, d, V, P = 300, 64, 3000, 1024
+    _, lm, t = random_case(T, d, V, P, 12)
+    x = np.zeros((T, d), np.uint16)
+    g = run_path(x, lm, t, P, 0)
+    assert abs(g["loss"] - np.log(P)) <= 1e-6 * np.log(P)
+    assert np.max(np.abs(g["lse"] - np.log(P))) <= 1e-5
+
+
+def test_deterministic():
+    x, lm, t = random_case(1000, 200, 5003, 3000, 13)
+    a = run_path(x, lm, t, 3000, 17)
+    b = run_path(x, lm, t, 3000, 17)
+    assert a["loss"] == b["loss"]
+    assert np.array_equal(a["lse"], b["lse"])
+    assert np.array_equal(a["dx_bits"], b["dx_bits"])
+    assert np.array_equal(a["dW_bits"], b["dW_bits"])
+
+
+def test_kernel_timing_records_every_kernel():
+    x, lm, t = random_case(512, 128, 5000, 1024, 14)
+    capi.ss_timing_reset()
+    capi.ss_timing_enable(True)
+    try:
+        run_path(x, lm, t, 1024, 0)
+    finally:
+        capi.ss_timing_enable(False)
+    rec = capi.ss_timing_read()
+    capi.ss_timing_reset()
+    for k in ("build_mark", "build_emit", "gather", "fwd_gemm_ce", "lse_combine", "loss_finalize",
+              "dlogits", "zero_rows", "dx_gemm", "dw_gemm_scatter"):
+        assert rec[k][0] == 1 and rec[k][1] > 0, (k, rec)
+
+
+# ------------------------------------------------ full-size workloads --
+
+def _sample(n, k, rng):
+    return np.sort(rng.choice(n, size=min(n, k), replace=False))
+
+
+@pytest.mark.parametrize("name", ["stage0", "stage2_early", "stage2_late", "full_softmax"])
+def test_full_size_workload(name):
+    w = wl.WORKLOADS[name]
+    x_bits, lm_bits, t = wl.workload_inputs(w)
+    g = run_path(x_bits, lm_bits, t, w.P, w.offset)
+    assert g["status"][0] == 0 and g["status"][8] == 0, g["status"]
+
+    cand, tpos, vpos, info = oc.build_candidates(t, w.V, w.P, w.offset)
+    assert np.array_equal(g["candidates"], cand)
+    assert np.array_equal(g["target_pos"], tpos)
+    assert np.array_equal(g["vocab_pos"], vpos)
+
+    x = wl.bits_to_f64(x_bits)
+    w_c = oc.gather_rows(wl.bits_to_f64(lm_bits), cand)
+    loss, lse, _, n = oc.sampled_ce_forward(x, w_c, tpos)
+    assert g["n_valid"] == n
+    assert abs(g["loss"] - loss) <= LOSS_RTOL * abs(loss), (g["loss"], loss)
+    assert np.max(np.abs(g["lse"] - lse)) <= LSE_ATOL
+
+    rng = np.random.default_rng(w.seed + 100)
+    scale = 1.0 / n
+    rows = _sample(w.T, 384, rng)
+    dx_o = oc.dx_rows(x[rows], w_c, tpos[rows], lse[rows], scale)
+    dx_g = wl.bits_to_f64(g["dx_bits"][rows])
+    assert rel_fro(dx_g, dx_o) <= GRAD_RTOL, rel_fro(dx_g, dx_o)
+
+    cols = np.unique(np.concatenate([_sample(w.P, 256, rng), tpos[tpos >= 0][:32]]))
+    dw_o = oc.dw_c_rows(x, w_c, tpos, lse, scale, cols)
+    dw_g = wl.bits_to_f64(g["dW_bits"][cand[cols]])
+    assert rel_fro(dw_g, dw_o) <= GRAD_RTOL, rel_fro(dw_g, dw_o)
+
+    in_c = np.zeros(w.V, bool)
+    in_c[cand] = True
+    assert np.all(g["dW_bits"][~in_c] == 0)
+    assert np.all(g["dx_bits"][tpos < 0] == 0)
