@@ -30,6 +30,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from sampled_softmax_cross_b200 import ranks  # noqa: E402
 from sampled_softmax_cross_b200 import workloads as wl  # noqa: E402
 
 METRIC = "tokens/s fused sampled-CE fwd+bwd at P=24576,d=768; % of BF16 tensor peak"
@@ -247,8 +248,9 @@ def run_ours(args, w):
     capi.load()
 
     # this rank's microbatch: own seed, staggered window start
-    x_bits, lm_bits, targets = wl.make_inputs(w.T, w.d, w.V, w.zipf_s, w.ignore_frac, w.seed + rank)
-    offset = (w.offset + (w.V * rank) // world) % w.V
+    x_bits, lm_bits, targets = wl.make_inputs(w.T, w.d, w.V, w.zipf_s, w.ignore_frac,
+                                              ranks.rank_seed(w.seed, rank))
+    offset = ranks.rank_offset(w.offset, w.V, rank, world)
     x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
     lm = torch.from_numpy(lm_bits.view(np.int16)).view(torch.bfloat16).to(dev)
     t = torch.from_numpy(targets).to(dev)
@@ -289,10 +291,7 @@ def run_ours(args, w):
     capi.ss_timing_reset()
     launches = sum(n for n, _ in kernels.values())
 
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = ranks.max_over_ranks(ms, dist if world > 1 else None, dev)
 
     # e2e: the same step from pinned host buffers, copies inside the timed region
     e2e = None
@@ -324,14 +323,12 @@ def run_ours(args, w):
         ev1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e_ms = torch.tensor([ev0.elapsed_time(ev1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e_ms = ranks.max_over_ranks(ev0.elapsed_time(ev1), dist if world > 1 else None, dev)
         h2d = hx.numel() * 2 + hlm.numel() * 2 + ht.numel() * 4
         d2h = 4 + hdx.numel() * 2 + hdW.numel() * 2
-        e2e = {"value": w.T * world * k2 / (float(e_ms.item()) / 1e3), "unit": "tokens/s",
+        e2e = {"value": w.T * world * k2 / (e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": float(e_ms.item()) / k2}
+               "ms_per_step": e_ms / k2}
 
     if rank == 0:
         pk = peaks()
