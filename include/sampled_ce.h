@@ -108,6 +108,30 @@ SS_API ss_status ss_build_candidates(const int32_t* targets, int64_t T, int32_t 
                               int32_t* target_pos, int32_t* vocab_pos, int32_t* dev_status,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* Allocation-free variant of ss_build_candidates. The pages the method comes
+ * from have no counterpart: it exists for callers that cannot give the
+ * library a workspace -- callers whose device memory is fixed once their
+ * set-up ends (a server or trainer whose caching allocator already holds all
+ * the memory it may use, a hook that must not allocate). They own the input
+ * and output arrays but cannot provide the extra scratch buffers.
+ * Same arguments (minus the workspace), results and dev_status as
+ * ss_build_candidates. The call allocates nothing: the bitmap and prefix
+ * scratch lives in a fixed 128 KB array inside the library, sized for
+ * V <= SS_MAX_VOCAB (a larger V returns SS_ERR_INVALID_ARG), present on every
+ * GPU that loads the library until the process exits.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. All calls on a device share the one array:
+ * calls whose work overlaps on the GPU (two streams, or two host threads
+ * without ordering) race and give wrong results, so order them on one
+ * stream. Each call rewrites every part of the array it reads, so nothing
+ * needs clearing between calls. */
+SS_API ss_status ss_build_candidates_noalloc(const int32_t* targets, int64_t T, int32_t V,
+                                             int32_t P, int64_t offset, int32_t stride,
+                                             int32_t* candidates, int32_t* target_pos,
+                                             int32_t* vocab_pos, int32_t* dev_status,
+                                             void* stream);
+
 /* Forward: W_C = lm_head[C] (sampled_softmax.py, SampledSoftmax._gather_rows),
  * logits z = x @ W_C^T with fp32 accumulation, and an online-softmax
  * cross-entropy over the P columns ("Learning Triton One Kernel at a Time:

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsampled_ce.so")
-SOURCES = ["ss_api.cu", "ce_kernels.cu", "ce_gemm.cu"]
+SOURCES = ["ss_api.cu", "ce_kernels.cu", "ce_gemm.cu", "ss_noalloc.cu"]
 HEADERS = ["sm100.cuh", "ss_internal.h"]
 
 NVCC_FLAGS = [

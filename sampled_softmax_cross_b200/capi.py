@@ -29,7 +29,8 @@ STATUS_NAMES = {
 STATUS = {v: k for k, v in STATUS_NAMES.items()}
 
 EXPORTS = (
-    "ss_workspace_bytes", "ss_build_workspace_bytes", "ss_build_candidates", "ss_ce_forward", "ss_ce_backward",
+    "ss_workspace_bytes", "ss_build_workspace_bytes", "ss_build_candidates",
+    "ss_build_candidates_noalloc", "ss_ce_forward", "ss_ce_backward",
     "ss_status_string", "ss_last_cuda_error", "ss_version", "ss_timing_enable",
     "ss_timing_reset", "ss_timing_count", "ss_timing_query",
 )
@@ -68,6 +69,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ss_workspace_bytes": (_sz, [_i64, _i32, _i32, _i32]),
         "ss_build_workspace_bytes": (_sz, [_i32]),
         "ss_build_candidates": (_i32, [_p, _i64, _i32, _i32, _i64, _i32, _p, _p, _p, _p, _p, _sz, _p]),
+        "ss_build_candidates_noalloc": (_i32, [_p, _i64, _i32, _i32, _i64, _i32, _p, _p, _p, _p,
+                                                _p]),
         "ss_ce_forward": (_i32, [_p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _p, _sz, _p]),
         "ss_ce_backward": (_i32, [_p, _p, _p, _p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p,
                                   _p, _sz, _p]),
@@ -127,6 +130,16 @@ def ss_build_candidates(targets, V, P, offset, stride, candidates, target_pos, v
         _ptr(vocab_pos), _ptr(dev_status), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream))
     _check("ss_build_candidates", code)
+
+
+def ss_build_candidates_noalloc(targets, V, P, offset, stride, candidates, target_pos,
+                                vocab_pos, dev_status, stream=None):
+    """ss_build_candidates without a workspace (scratch inside the library)."""
+    T = targets.numel()
+    code = load().ss_build_candidates_noalloc(
+        _ptr(targets), T, V, P, offset, stride, _ptr(candidates), _ptr(target_pos),
+        _ptr(vocab_pos), _ptr(dev_status), _stream(stream))
+    _check("ss_build_candidates_noalloc", code)
 
 
 def ss_ce_forward(x, lm_head, candidates, target_pos, T, d, V, P, loss, lse, n_valid, dev_status,
