@@ -340,11 +340,9 @@ def run_ours(args, w):
             "fwd_gemm_ce": ("tensor", flops_gemm), "dx_gemm": ("tensor", flops_gemm),
             "dw_gemm_scatter": ("tensor", flops_gemm),
             "gather": ("hbm", 2.0 * w.P * w.d * 2),
-            "dlogits": ("hbm", 2.0 * w.T * w.P * 2),
             "zero_rows": ("hbm", (w.V - w.P) * w.d * 2.0 + w.V * 4),
             "build_mark": ("hbm", w.T * 4.0 + 2 * ((w.V + 31) // 32) * 4),
             "build_emit": ("hbm", w.T * 4.0 * 2 + w.V * 4.0 * 2 + w.P * 4.0),
-            "lse_combine": ("hbm", ((w.P + 255) // 256) * w.T * 8.0 + w.T * 16.0),
         }
         total_k = sum(t for _, t in kernels.values())
         for k, (n, tot) in kernels.items():

@@ -72,7 +72,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ss_build_candidates_noalloc": (_i32, [_p, _i64, _i32, _i32, _i64, _i32, _p, _p, _p, _p,
                                                 _p]),
         "ss_ce_forward": (_i32, [_p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _p, _sz, _p]),
-        "ss_ce_backward": (_i32, [_p, _p, _p, _p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p,
+        "ss_ce_backward": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p,
                                   _p, _sz, _p]),
         "ss_status_string": (ctypes.c_char_p, [_i32]),
         "ss_last_cuda_error": (ctypes.c_char_p, []),
@@ -151,10 +151,10 @@ def ss_ce_forward(x, lm_head, candidates, target_pos, T, d, V, P, loss, lse, n_v
     _check("ss_ce_forward", code)
 
 
-def ss_ce_backward(grad_loss, x, candidates, target_pos, vocab_pos, lse, n_valid, T, d, V, P, dx,
+def ss_ce_backward(grad_loss, x, candidates, target_pos, vocab_pos, n_valid, T, d, V, P, dx,
                    dW, dev_status, workspace, stream=None):
     code = load().ss_ce_backward(
-        _ptr(grad_loss), _ptr(x), _ptr(candidates), _ptr(target_pos), _ptr(vocab_pos), _ptr(lse),
+        _ptr(grad_loss), _ptr(x), _ptr(candidates), _ptr(target_pos), _ptr(vocab_pos),
         _ptr(n_valid), T, d, V, P, _ptr(dx), _ptr(dW), _ptr(dev_status), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check("ss_ce_backward", code)
@@ -231,7 +231,7 @@ class SampledCE:
 
     def backward(self, x, grad_loss=None, stream=None):
         g = self.grad_loss if grad_loss is None else grad_loss
-        ss_ce_backward(g, x, self.candidates, self.target_pos, self.vocab_pos, self.lse,
+        ss_ce_backward(g, x, self.candidates, self.target_pos, self.vocab_pos,
                        self.n_valid, self.T, self.d, self.V, self.P, self.dx, self.dW,
                        self.dev_status, self.workspace, stream)
 

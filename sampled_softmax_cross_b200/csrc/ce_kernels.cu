@@ -1,14 +1,12 @@
 // ce_kernels.cu -- the memory- and latency-bound steps of the sampled-softmax
-// CE head: candidate build, row gather, LSE combine / loss reduction, dlogits
-// and the zero rows of the dense lm_head gradient.
+// CE head: candidate build, row gather, the final loss reduction and the zero
+// rows of the dense lm_head gradient.
 #include <limits.h>
 
 #include "sm100.cuh"
 #include "ss_internal.h"
 
 namespace ssb {
-
-constexpr float kLog2e = 1.4426950408889634f;
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 constexpr int kBuildThreads = 1024;
@@ -248,10 +246,15 @@ __global__ void k_build_emit(const int32_t* __restrict__ targets, int64_t T, int
 // Row gather W_C[j] = lm_head[C_j] (sampled_softmax.py, _gather_rows): one warp
 // per row, 16-byte vectors.
 // ----------------------------------------------------------------------------
+// Block 0 also clears `zero_words` (the forward's tile counters) for the
+// kernel that follows on the stream.
 __global__ void k_gather(const uint4* __restrict__ lm, const int32_t* __restrict__ cand, int32_t P,
                          int32_t vec_per_row, int32_t V, uint4* __restrict__ w_c,
-                         int32_t* __restrict__ status) {
+                         int32_t* __restrict__ status, int32_t* __restrict__ zero_words,
+                         int32_t n_zero_words) {
   const int lane = threadIdx.x & 31;
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero_words; i += blockDim.x) zero_words[i] = 0;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < P; r += warps) {
     const int c = __ldg(cand + r);
@@ -274,64 +277,14 @@ __global__ void k_gather(const uint4* __restrict__ lm, const int32_t* __restrict
 }
 
 // ----------------------------------------------------------------------------
-// LSE combine: merge the per-tile (max, sum) pairs of each row; per-row loss;
-// per-block partial sums in a fixed order (deterministic).
+// Loss: sum the per-work-item (loss sum, valid rows) pairs the forward's
+// converter warps wrote, in item order (deterministic), and divide.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(kCombineThreads)
-    k_combine(const float2* __restrict__ stats, const float* __restrict__ zt,
-              const int32_t* __restrict__ tpos, int64_t T, int32_t P, int32_t tiles_n,
-              float* __restrict__ lse, double* __restrict__ partials) {
-  __shared__ double s_sum[kCombineThreads / 32];
-  __shared__ int s_cnt[kCombineThreads / 32];
-  const int64_t i = (int64_t)blockIdx.x * kCombineThreads + threadIdx.x;
-  double my = 0.0;
-  int cnt = 0;
-  if (i < T) {
-    float M = -INFINITY, S = 0.f;
-    for (int n = 0; n < tiles_n; ++n) {
-      const float2 p = stats[(int64_t)n * T + i];
-      if (p.x > M) {
-        S = S * ex2_approx((M - p.x) * kLog2e) + p.y;
-        M = p.x;
-      } else {
-        S += p.y * ex2_approx((p.x - M) * kLog2e);
-      }
-    }
-    const float l = M + logf(S);
-    lse[i] = l;
-    const int t = tpos[i];
-    if (t >= 0 && t < P) {
-      my = (double)l - (double)zt[i];
-      cnt = 1;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    my += __shfl_down_sync(0xffffffffu, my, o);
-    cnt += __shfl_down_sync(0xffffffffu, cnt, o);
-  }
-  if ((threadIdx.x & 31) == 0) {
-    s_sum[threadIdx.x >> 5] = my;
-    s_cnt[threadIdx.x >> 5] = cnt;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double s = 0.0;
-    int c = 0;
-    for (int w = 0; w < kCombineThreads / 32; ++w) {
-      s += s_sum[w];
-      c += s_cnt[w];
-    }
-    partials[2 * blockIdx.x] = s;
-    partials[2 * blockIdx.x + 1] = (double)c;
-  }
-}
-
-__global__ void k_finalize(const double* __restrict__ partials, int32_t nblocks,
+__global__ void k_finalize(const double* __restrict__ partials, int32_t nitems,
                            float* __restrict__ loss, int32_t* __restrict__ n_valid) {
   __shared__ double s_sum[32], s_cnt[32];
   double s = 0.0, c = 0.0;
-  for (int b = threadIdx.x; b < nblocks; b += blockDim.x) {
+  for (int b = threadIdx.x; b < nitems; b += blockDim.x) {
     s += partials[2 * b];
     c += partials[2 * b + 1];
   }
@@ -353,59 +306,6 @@ __global__ void k_finalize(const double* __restrict__ partials, int32_t nblocks,
     }
     *n_valid = (int32_t)tc;
     *loss = tc > 0.0 ? (float)(ts / tc) : 0.f;
-  }
-}
-
-// ----------------------------------------------------------------------------
-// dlogits in place: G = (g / n) (exp(z - lse) - onehot), 0 on ignored rows
-// ("Learning Triton ... Softmax", section "Gradient").
-// ----------------------------------------------------------------------------
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__global__ void __launch_bounds__(256)
-    k_dlogits(uint16_t* __restrict__ z, int64_t T, int32_t P, int64_t ldz,
-              const float* __restrict__ lse, const int32_t* __restrict__ tpos,
-              const float* __restrict__ grad_loss, const int32_t* __restrict__ n_valid) {
-  const int nv = *n_valid;
-  const float coef = nv > 0 ? *grad_loss / (float)nv : 0.f;
-  const int vpr = (int)(ldz >> 3);  // 16-byte vectors per row
-  for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
-    uint4* zr = reinterpret_cast<uint4*>(z + row * ldz);
-    const int t = __ldg(tpos + row);
-    if (t < 0 || t >= P || coef == 0.f) {
-      for (int v = threadIdx.x; v < vpr; v += blockDim.x) __stcs(zr + v, make_uint4(0, 0, 0, 0));
-      continue;
-    }
-    const float l2 = __ldg(lse + row) * kLog2e;
-    for (int v0 = threadIdx.x; v0 < vpr; v0 += 4 * blockDim.x) {
-      uint4 in[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int v = v0 + u * blockDim.x;
-        if (v < vpr) in[u] = __ldcs(zr + v);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int v = v0 + u * blockDim.x;
-        if (v < vpr) {
-          const uint32_t w[4] = {in[u].x, in[u].y, in[u].z, in[u].w};
-          uint32_t o[4];
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const int c = v * 8 + 2 * h;
-            float a = coef * ex2_approx(fmaf(bf16_lo(w[h]), kLog2e, -l2));
-            float b = coef * ex2_approx(fmaf(bf16_hi(w[h]), kLog2e, -l2));
-            if (c == t) a -= coef;
-            if (c + 1 == t) b -= coef;
-            if (c >= P) a = 0.f;
-            if (c + 1 >= P) b = 0.f;
-            o[h] = pack_bf16x2(a, b);
-          }
-          __stcs(zr + v, make_uint4(o[0], o[1], o[2], o[3]));
-        }
-      }
-    }
   }
 }
 
@@ -463,35 +363,20 @@ cudaError_t launch_build_emit(const int32_t* targets, int64_t T, int32_t V, int3
 }
 
 cudaError_t launch_gather(const uint16_t* lm_head, const int32_t* cand, int32_t P, int32_t d,
-                          int32_t V, uint16_t* w_c, int32_t* status, cudaStream_t s) {
+                          int32_t V, uint16_t* w_c, int32_t* status, int32_t* zero_words,
+                          int32_t n_zero_words, cudaStream_t s) {
   const int warps_per_block = 8;
   const int blocks = (int)min64((P + warps_per_block - 1) / warps_per_block,
                                        (int64_t)num_sms() * 16);
   k_gather<<<blocks, warps_per_block * 32, 0, s>>>(reinterpret_cast<const uint4*>(lm_head), cand, P,
-                                                    d / 8, V, reinterpret_cast<uint4*>(w_c), status);
+                                                    d / 8, V, reinterpret_cast<uint4*>(w_c), status,
+                                                    zero_words, n_zero_words);
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const float2* stats, const float* zt, const int32_t* tpos, int64_t T,
-                           int32_t P, int32_t tiles_n, float* lse, double* partials,
-                           int32_t nblocks, cudaStream_t s) {
-  if (nblocks == 0) return cudaSuccess;
-  k_combine<<<nblocks, kCombineThreads, 0, s>>>(stats, zt, tpos, T, P, tiles_n, lse, partials);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_finalize(const double* partials, int32_t nblocks, float* loss,
+cudaError_t launch_finalize(const double* partials, int32_t nitems, float* loss,
                             int32_t* n_valid, cudaStream_t s) {
-  k_finalize<<<1, 1024, 0, s>>>(partials, nblocks, loss, n_valid);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_dlogits(uint16_t* z, int64_t T, int32_t P, int64_t ldz, const float* lse,
-                           const int32_t* tpos, const float* grad_loss, const int32_t* n_valid,
-                           cudaStream_t s) {
-  if (T == 0) return cudaSuccess;
-  const int blocks = (int)min64(T, (int64_t)num_sms() * 8);
-  k_dlogits<<<blocks, 256, 0, s>>>(z, T, P, ldz, lse, tpos, grad_loss, n_valid);
+  k_finalize<<<1, 1024, 0, s>>>(partials, nitems, loss, n_valid);
   return cudaGetLastError();
 }
 

@@ -112,6 +112,116 @@ SS_DEV void bulk_wait() {
 // Make generic-proxy writes to shared memory visible to the async proxy (TMA).
 SS_DEV void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// Order completed async-proxy (TMA) global writes before later generic accesses.
+SS_DEV void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Wait until at most `n` bulk groups of this thread are pending (n in 0..4).
+SS_DEV void bulk_wait_at_most(int n) {
+  switch (n) {
+    case 0: bulk_wait<0>(); break;
+    case 1: bulk_wait<1>(); break;
+    case 2: bulk_wait<2>(); break;
+    case 3: bulk_wait<3>(); break;
+    default: bulk_wait<4>(); break;
+  }
+}
+
+// Named barrier over `nthreads` threads (id 0 is __syncthreads).
+SS_DEV void named_barrier(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier that also returns, to every participant, whether any of
+// them passed `pred` = true (a uniform decision for a group of warps).
+SS_DEV bool named_barrier_any(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)(pred ? 1 : 0)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+SS_DEV int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+SS_DEV int ld_acquire_cta_shared(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+
+SS_DEV void red_release_cta_shared_add(int* p, int v) {
+  asm volatile("red.release.cta.shared::cta.add.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v)
+               : "memory");
+}
+
+SS_DEV void red_release_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait (whole warp) until *ctr >= target; false on abort or after the time limit.
+SS_DEV bool wait_counter(const int* ctr, int target, const volatile int* abort_flag) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) {
+    const unsigned long long t0 = globaltimer();
+    while (ld_acquire(ctr) < target) {
+      if (*abort_flag || globaltimer() - t0 > kWaitLimitNs) {
+        ok = false;
+        break;
+      }
+      __nanosleep(200);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok) (void)ld_acquire(ctr);  // every lane acquires before reading the data
+  return ok;
+}
+
+// ----------------------------------------------------------------- cluster --
+
+SS_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory offset in CTA `rank`.
+SS_DEV uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+SS_DEV void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+
+// Arrive on an mbarrier given by its shared::cluster address (may be the peer's).
+SS_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+// 2-D tiled load into this CTA's shared memory whose completion is counted on
+// an mbarrier of the CTA pair's leader (shared::cluster address). No multicast.
+SS_DEV void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster_addr,
+                             int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y)
+      : "memory");
+}
+
 // ----------------------------------------------------------- tcgen05 / TMEM --
 
 SS_DEV void tmem_alloc(uint32_t* holder, uint32_t ncols) {  // whole warp
@@ -149,6 +259,44 @@ SS_DEV void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// CTA-pair forms (cta_group::2): the pair's leader issues the MMA for a
+// 256-row tile whose A rows and B columns are split across the two CTAs.
+SS_DEV void tmem_alloc_pair(uint32_t* holder, uint32_t ncols) {  // one warp in each CTA
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(holder)),
+               "r"(ncols)
+               : "memory");
+}
+
+SS_DEV void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+SS_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+SS_DEV void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the mbarrier at this shared-memory offset in every CTA of
+// `cta_mask` once the MMAs issued so far by this thread have completed.
+SS_DEV void umma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
 }
 
 SS_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

@@ -31,12 +31,13 @@ ss_status cuda_fail(cudaError_t e, const char* where) {
 struct DeviceState {
   bool ready = false;
   int sms = 0;
+  int max_pairs[3] = {0, 0, 0};  // resident CTA pairs of each GEMM kernel
   ss_status status = SS_OK;
 };
 std::mutex g_dev_mu;
 DeviceState g_dev[128];
 
-ss_status ensure_device(int* sms) {
+ss_status ensure_device(int* sms, int* max_pairs = nullptr) {
   int dev = 0;
   SS_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev < 0 || dev >= 128) return SS_ERR_UNSUPPORTED_DEVICE;
@@ -51,15 +52,19 @@ ss_status ensure_device(int* sms) {
     if (major != 10) {
       d.status = SS_ERR_UNSUPPORTED_DEVICE;
     } else {
-      for (int k = 0; k < 3; ++k)
+      for (int k = 0; k < 3; ++k) {
         SS_CUDA(cudaFuncSetAttribute(gemm_kernel_ptr(k),
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      gemm_smem_bytes()),
                 "cudaFuncSetAttribute");
+        d.max_pairs[k] = gemm_max_pairs(k, d.sms);
+      }
     }
     d.ready = true;
   }
   *sms = d.sms;
+  if (max_pairs != nullptr)
+    for (int k = 0; k < 3; ++k) max_pairs[k] = d.max_pairs[k];
   return d.status;
 }
 
@@ -143,15 +148,16 @@ void timing_end(int slot, cudaStream_t s) {
   } while (0)
 
 // -------------------------------------------------------------- workspace --
-constexpr int kBM = 128, kBN = 256;
+constexpr int kBM = 128, kBN = 256, kBMP = 256;  // rows per CTA, cols per tile, rows per pair
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-  size_t bitmap, prefix, partials, w_c, z, stats, zt, total;
+  size_t bitmap, prefix, partials, counters, w_c, z, stats, zt, total;
   int64_t ldz;
   int tiles_n;
-  int nblk;
+  int nitems;   // converter work items (kRowsPerItem rows each)
+  int nhalf;    // 128-row half-stripes of all pair tiles; counters = nhalf + 1 ticket
 };
 
 bool sizes_ok(int64_t T, int32_t d, int32_t V, int32_t P) {
@@ -164,14 +170,17 @@ Layout layout(int64_t T, int32_t d, int32_t V, int32_t P) {
   const size_t nw = (size_t)(V + 31) / 32;
   L.ldz = (P + 7) / 8 * 8;
   L.tiles_n = (P + kBN - 1) / kBN;
-  L.nblk = combine_blocks(T);
+  L.nitems = converter_items(T);
+  L.nhalf = 2 * (int)((T + kBMP - 1) / kBMP);  // both CTAs of every pair tile publish
   size_t off = 0;
   L.bitmap = off;
   off += align_up(nw * 4, 256);
   L.prefix = off;
   off += align_up(nw * 4, 256);
   L.partials = off;
-  off += align_up((size_t)L.nblk * 16 + 16, 256);
+  off += align_up((size_t)L.nitems * 16 + 16, 256);
+  L.counters = off;
+  off += align_up((size_t)(L.nhalf + 1) * 4, 256);
   off = align_up(off, 1024);
   L.w_c = off;
   off += align_up((size_t)P * d * 2, 1024);
@@ -275,8 +284,8 @@ ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t*
     return SS_ERR_MISALIGNED;
   const Layout L = layout(T, d, V, P);
   if (workspace_bytes < L.total) return SS_ERR_WORKSPACE_TOO_SMALL;
-  int sms;
-  ss_status ds = ensure_device(&sms);
+  int sms, pairs[3];
+  ss_status ds = ensure_device(&sms, pairs);
   if (ds != SS_OK) return ds;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -285,51 +294,59 @@ ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t*
   float2* stats = reinterpret_cast<float2*>(ws + L.stats);
   float* zt = reinterpret_cast<float*>(ws + L.zt);
   double* partials = reinterpret_cast<double*>(ws + L.partials);
+  int32_t* counters = reinterpret_cast<int32_t*>(ws + L.counters);
   int32_t* kstatus = dev_status + 8;
 
-  SS_LAUNCH("gather", s, launch_gather(lm_head, candidates, P, d, V, w_c, kstatus, s));
+  SS_LAUNCH("gather", s,
+            launch_gather(lm_head, candidates, P, d, V, w_c, kstatus, counters, L.nhalf + 1, s));
   if (T > 0) {
     CUtensorMap ta, tb, tc;
     ss_status r;
     if ((r = make_map(&ta, x, d, T, d, 64, kBM)) != SS_OK) return r;
-    if ((r = make_map(&tb, w_c, d, P, d, 64, kBN)) != SS_OK) return r;
+    if ((r = make_map(&tb, w_c, d, P, d, 64, kBN / 2)) != SS_OK) return r;
     if ((r = make_map(&tc, z, P, T, L.ldz, 64, 32)) != SS_OK) return r;
     GemmArgs a{};
     a.M = (int32_t)T;
     a.N = P;
     a.K = d;
-    a.tiles_m = (int32_t)((T + kBM - 1) / kBM);
+    a.tiles_m = (int32_t)((T + kBMP - 1) / kBMP);
     a.tiles_n = L.tiles_n;
     a.num_kb = (d + 63) / 64;
     a.tpos = target_pos;
     a.stats = stats;
     a.zt = zt;
+    a.u = z;
+    a.ldz = L.ldz;
+    a.done = counters;
+    a.ticket = counters + L.nhalf;
+    a.lse = lse;
+    a.partials = partials;
+    a.num_items = L.nitems;
     a.status = kstatus;
     const int tiles = a.tiles_m * a.tiles_n;
-    SS_LAUNCH("fwd_gemm_ce", s, launch_gemm(KIND_FWD, ta, tb, tc, a, tiles < sms ? tiles : sms, s));
-    SS_LAUNCH("lse_combine", s,
-              launch_combine(stats, zt, target_pos, T, P, L.tiles_n, lse, partials, L.nblk, s));
+    SS_LAUNCH("fwd_gemm_ce", s,
+              launch_gemm(KIND_FWD, ta, tb, tc, a, tiles < pairs[KIND_FWD] ? tiles : pairs[KIND_FWD], s));
   }
-  SS_LAUNCH("loss_finalize", s, launch_finalize(partials, L.nblk, loss, n_valid, s));
+  SS_LAUNCH("loss_finalize", s, launch_finalize(partials, T > 0 ? L.nitems : 0, loss, n_valid, s));
   return SS_OK;
 }
 
 ss_status ss_ce_backward(const float* grad_loss, const ss_bf16* x, const int32_t* candidates,
-                         const int32_t* target_pos, const int32_t* vocab_pos, const float* lse,
+                         const int32_t* target_pos, const int32_t* vocab_pos,
                          const int32_t* n_valid, int64_t T, int32_t d, int32_t V, int32_t P,
                          ss_bf16* dx, ss_bf16* dW, int32_t* dev_status, void* workspace,
                          size_t workspace_bytes, void* stream) {
   if (!sizes_ok(T, d, V, P)) return SS_ERR_INVALID_ARG;
   if (grad_loss == nullptr || candidates == nullptr || vocab_pos == nullptr ||
       n_valid == nullptr || dW == nullptr || dev_status == nullptr || workspace == nullptr ||
-      (T > 0 && (x == nullptr || target_pos == nullptr || lse == nullptr || dx == nullptr)))
+      (T > 0 && (x == nullptr || target_pos == nullptr || dx == nullptr)))
     return SS_ERR_INVALID_ARG;
   if (!aligned16(dW) || !aligned16(workspace) || (T > 0 && (!aligned16(x) || !aligned16(dx))))
     return SS_ERR_MISALIGNED;
   const Layout L = layout(T, d, V, P);
   if (workspace_bytes < L.total) return SS_ERR_WORKSPACE_TOO_SMALL;
-  int sms;
-  ss_status ds = ensure_device(&sms);
+  int sms, pairs[3];
+  ss_status ds = ensure_device(&sms, pairs);
   if (ds != SS_OK) return ds;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -341,41 +358,46 @@ ss_status ss_ce_backward(const float* grad_loss, const ss_bf16* x, const int32_t
     SS_LAUNCH("zero_rows", s, launch_zero_rows(dW, V, d, vocab_pos, 1, s));
     return SS_OK;
   }
-  SS_LAUNCH("dlogits", s, launch_dlogits(z, T, P, L.ldz, lse, target_pos, grad_loss, n_valid, s));
   SS_LAUNCH("zero_rows", s, launch_zero_rows(dW, V, d, vocab_pos, 0, s));
 
   CUtensorMap ga, wb, dxs, ga2, xb;
   ss_status r;
-  if ((r = make_map(&ga, z, P, T, L.ldz, 64, kBM)) != SS_OK) return r;   // G, K-major
+  if ((r = make_map(&ga, z, P, T, L.ldz, 64, kBM)) != SS_OK) return r;   // U, K-major
   if ((r = make_map(&wb, w_c, d, P, d, 64, 64)) != SS_OK) return r;      // W_C, MN-major
   if ((r = make_map(&dxs, dx, d, T, d, 64, 32)) != SS_OK) return r;      // dx store
-  if ((r = make_map(&ga2, z, P, T, L.ldz, 64, 64)) != SS_OK) return r;   // G^T, MN-major
+  if ((r = make_map(&ga2, z, P, T, L.ldz, 64, 64)) != SS_OK) return r;   // U^T, MN-major
   if ((r = make_map(&xb, x, d, T, d, 64, 64)) != SS_OK) return r;        // x, MN-major
 
   GemmArgs a{};
   a.M = (int32_t)T;
   a.N = d;
   a.K = P;
-  a.tiles_m = (int32_t)((T + kBM - 1) / kBM);
+  a.tiles_m = (int32_t)((T + kBMP - 1) / kBMP);
   a.tiles_n = (d + kBN - 1) / kBN;
   a.num_kb = (P + 63) / 64;
+  a.grad_loss = grad_loss;
+  a.n_valid = n_valid;
   a.status = kstatus;
   int tiles = a.tiles_m * a.tiles_n;
-  SS_LAUNCH("dx_gemm", s, launch_gemm(KIND_DX, ga, wb, dxs, a, tiles < sms ? tiles : sms, s));
+  SS_LAUNCH("dx_gemm", s,
+            launch_gemm(KIND_DX, ga, wb, dxs, a, tiles < pairs[KIND_DX] ? tiles : pairs[KIND_DX], s));
 
   GemmArgs b{};
   b.M = P;
   b.N = d;
   b.K = (int32_t)T;
-  b.tiles_m = (P + kBM - 1) / kBM;
+  b.tiles_m = (P + kBMP - 1) / kBMP;
   b.tiles_n = (d + kBN - 1) / kBN;
   b.num_kb = (int32_t)((T + 63) / 64);
   b.cand = candidates;
   b.dW = dW;
   b.V = V;
+  b.grad_loss = grad_loss;
+  b.n_valid = n_valid;
   b.status = kstatus;
   tiles = b.tiles_m * b.tiles_n;
-  SS_LAUNCH("dw_gemm_scatter", s, launch_gemm(KIND_DW, ga2, xb, ga2, b, tiles < sms ? tiles : sms, s));
+  SS_LAUNCH("dw_gemm_scatter", s,
+            launch_gemm(KIND_DW, ga2, xb, ga2, b, tiles < pairs[KIND_DW] ? tiles : pairs[KIND_DW], s));
   return SS_OK;
 }
 

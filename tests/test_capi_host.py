@@ -111,9 +111,9 @@ def test_forward_backward_host_rejections(lib):
     assert f(mis, a, a, a, 512, 128, 50304, 2048, a, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_MISALIGNED"]
     assert f(a, None, a, a, 512, 128, 50304, 2048, a, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
     b = lib.ss_ce_backward
-    assert b(a, a, a, a, a, a, a, 512, 128, 50304, 2049 * 0 + 50305, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
-    assert b(a, a, a, a, a, a, a, 512, 128, 50304, 2048, a, mis, a, a, ws, None) == capi.STATUS["SS_ERR_MISALIGNED"]
-    assert b(None, a, a, a, a, a, a, 512, 128, 50304, 2048, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    assert b(a, a, a, a, a, a, 512, 128, 50304, 50305, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    assert b(a, a, a, a, a, a, 512, 128, 50304, 2048, a, mis, a, a, ws, None) == capi.STATUS["SS_ERR_MISALIGNED"]
+    assert b(None, a, a, a, a, a, 512, 128, 50304, 2048, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
 
 
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
