@@ -77,7 +77,7 @@ typedef enum ss_status {
 /* Bytes of workspace the three calls need for these sizes (0 if the sizes
  * are invalid). One workspace serves ss_build_candidates, ss_ce_forward and
  * ss_ce_backward of the same microbatch; ss_ce_forward leaves the gathered
- * rows W_C and U (softmax minus one-hot) in it for ss_ce_backward, so it must not be
+ * rows W_C and the gradient factors (below) in it for ss_ce_backward, so it must not be
  * reused between a forward and its backward (the "one microbatch per step"
  * contract of sampled_softmax.py, SampledSoftmax.__init__). */
 SS_API size_t ss_workspace_bytes(int64_t T, int32_t d, int32_t V, int32_t P);
@@ -141,13 +141,15 @@ SS_API ss_status ss_build_candidates_noalloc(const int32_t* targets, int64_t T, 
  *             0 when n_valid = 0 (token-weighted mean, as in Handout #16's
  *             lm_gradient);
  *   n_valid = number of rows with target_pos >= 0.
- * The same kernel also forms the loss gradient w.r.t. the logits, up to the
- * scalar g / n_valid (section "Gradient": softmax minus one-hot):
- *   U_ij = exp(z_ij - lse_i) - [j == target_pos_i] on valid rows, 0 on ignored rows.
+ * The forward also leaves in the workspace what the backward needs for the
+ * loss gradient w.r.t. the logits (section "Gradient": softmax minus one-hot):
+ * E'_ij = exp(z_ij - z_i,target) (bf16; 1 - S_i at the target column, S_i the
+ * row sum), r_i = 1 / S_i and x'_i = r_i x_i, so that r_i E'_ij equals
+ * softmax_ij - [j == target_pos_i]; ignored rows have r_i = 0 and x'_i = 0.
  * In:  x [T, d] bf16; lm_head [V, d] bf16; candidates [P], target_pos [T] as
  *      written by ss_build_candidates. d % 8 == 0.
  * Out: loss [1] float32, lse [T] float32, n_valid [1] int32.
- * Workspace: keeps W_C [P, d] bf16 and U [T, P] bf16 for the backward. */
+ * Workspace: keeps W_C [P, d], E' [T, P] and x' [T, d] (bf16) for the backward. */
 SS_API ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t* candidates,
                         const int32_t* target_pos, int64_t T, int32_t d, int32_t V, int32_t P,
                         float* loss, float* lse, int32_t* n_valid, int32_t* dev_status,
@@ -155,19 +157,21 @@ SS_API ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const i
 
 /* Backward of the loss above for an upstream gradient g = grad_loss[0]
  * ("Learning Triton ... Softmax", section "Gradient": softmax minus one-hot):
- *   G     = (g / n_valid) * U  (0 everywhere when n_valid = 0), U from the forward;
+ *   G     = (g / n_valid) * (softmax - onehot)  (0 when n_valid = 0);
  *   dx    = G @ W_C                      [T, d] bf16;
  *   dW    = dense [V, d] bf16: row C_j = (G^T @ x)_j, every other row +0.0
  *           (module docstring: "dense over the vocabulary with zeros outside C").
- * In:  grad_loss [1] float32 (device); x, candidates, target_pos, vocab_pos as
- *      above; n_valid from ss_ce_forward; the workspace the forward used.
+ * Computed from the forward's workspace as dx = (g/n) r (.) (E' @ W_C) and
+ * dW_C = (g/n) E'^T @ x'.
+ * In:  grad_loss [1] float32 (device); candidates, vocab_pos as above; n_valid
+ *      from ss_ce_forward; the workspace the forward used (it holds the x' rows).
  * Out: dx [T, d], dW [V, d] (fully written). The workspace is only read, so
  *      the backward may be repeated (for another grad_loss) after one forward. */
-SS_API ss_status ss_ce_backward(const float* grad_loss, const ss_bf16* x, const int32_t* candidates,
-                         const int32_t* target_pos, const int32_t* vocab_pos,
-                         const int32_t* n_valid, int64_t T, int32_t d, int32_t V, int32_t P,
-                         ss_bf16* dx, ss_bf16* dW, int32_t* dev_status, void* workspace,
-                         size_t workspace_bytes, void* stream);
+SS_API ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
+                         const int32_t* vocab_pos, const int32_t* n_valid, int64_t T,
+                         int32_t d, int32_t V, int32_t P, ss_bf16* dx, ss_bf16* dW,
+                         int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                         void* stream);
 
 /* Human-readable name of a status code (static storage). */
 SS_API const char* ss_status_string(int32_t status);

@@ -72,8 +72,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ss_build_candidates_noalloc": (_i32, [_p, _i64, _i32, _i32, _i64, _i32, _p, _p, _p, _p,
                                                 _p]),
         "ss_ce_forward": (_i32, [_p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _p, _sz, _p]),
-        "ss_ce_backward": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p,
-                                  _p, _sz, _p]),
+        "ss_ce_backward": (_i32, [_p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _sz,
+                                  _p]),
         "ss_status_string": (ctypes.c_char_p, [_i32]),
         "ss_last_cuda_error": (ctypes.c_char_p, []),
         "ss_version": (_i32, []),
@@ -151,11 +151,10 @@ def ss_ce_forward(x, lm_head, candidates, target_pos, T, d, V, P, loss, lse, n_v
     _check("ss_ce_forward", code)
 
 
-def ss_ce_backward(grad_loss, x, candidates, target_pos, vocab_pos, n_valid, T, d, V, P, dx,
-                   dW, dev_status, workspace, stream=None):
+def ss_ce_backward(grad_loss, candidates, vocab_pos, n_valid, T, d, V, P, dx, dW, dev_status,
+                   workspace, stream=None):
     code = load().ss_ce_backward(
-        _ptr(grad_loss), _ptr(x), _ptr(candidates), _ptr(target_pos), _ptr(vocab_pos),
-        _ptr(n_valid), T, d, V, P, _ptr(dx), _ptr(dW), _ptr(dev_status), _ptr(workspace),
+        _ptr(grad_loss), _ptr(candidates), _ptr(vocab_pos), _ptr(n_valid), T, d, V, P, _ptr(dx), _ptr(dW), _ptr(dev_status), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check("ss_ce_backward", code)
 
@@ -229,16 +228,15 @@ class SampledCE:
         ss_ce_forward(x, lm_head, self.candidates, self.target_pos, self.T, self.d, self.V, self.P,
                       self.loss, self.lse, self.n_valid, self.dev_status, self.workspace, stream)
 
-    def backward(self, x, grad_loss=None, stream=None):
+    def backward(self, grad_loss=None, stream=None):
         g = self.grad_loss if grad_loss is None else grad_loss
-        ss_ce_backward(g, x, self.candidates, self.target_pos, self.vocab_pos,
-                       self.n_valid, self.T, self.d, self.V, self.P, self.dx, self.dW,
+        ss_ce_backward(g, self.candidates, self.vocab_pos, self.n_valid, self.T, self.d, self.V, self.P, self.dx, self.dW,
                        self.dev_status, self.workspace, stream)
 
     def step(self, targets, x, lm_head, offset, stride=DEFAULT_STRIDE, grad_loss=None, stream=None):
         self.build(targets, offset, stride, stream)
         self.forward(x, lm_head, stream)
-        self.backward(x, grad_loss, stream)
+        self.backward(grad_loss, stream)
 
     def status(self) -> list[int]:
         return self.dev_status.tolist()

@@ -1,6 +1,8 @@
 // ce_kernels.cu -- the memory- and latency-bound steps of the sampled-softmax
-// CE head: candidate build, row gather, the final loss reduction and the zero
-// rows of the dense lm_head gradient.
+// CE head: candidate build, row gather, reference logits, the row pass after
+// the forward GEMM (lse, loss terms, gradient scales), the exact fix-up of
+// overflowing rows, the loss reduction and the zero rows of the dense
+// lm_head gradient.
 #include <limits.h>
 
 #include "sm100.cuh"
@@ -277,16 +279,177 @@ __global__ void k_gather(const uint4* __restrict__ lm, const int32_t* __restrict
 }
 
 // ----------------------------------------------------------------------------
-// Loss: sum the per-work-item (loss sum, valid rows) pairs the forward's
-// converter warps wrote, in item order (deterministic), and divide.
+// Reference logit per row: ref_i = x_i . W_C[target_pos_i] in fp32 (W_C[0] on
+// ignored rows). The forward GEMM's epilogue stores exp(z - ref) (ce_gemm.cu).
+// One warp per row; fixed summation order.
 // ----------------------------------------------------------------------------
-__global__ void k_finalize(const double* __restrict__ partials, int32_t nitems,
-                           float* __restrict__ loss, int32_t* __restrict__ n_valid) {
+__device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
+  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    acc = fmaf(__uint_as_float(wa[h] << 16), __uint_as_float(wb[h] << 16), acc);
+    acc = fmaf(__uint_as_float(wa[h] & 0xffff0000u), __uint_as_float(wb[h] & 0xffff0000u), acc);
+  }
+  return acc;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+  return __shfl_sync(0xffffffffu, v, 0);
+}
+
+__global__ void k_ref_logits(const uint4* __restrict__ x, const uint4* __restrict__ w_c,
+                             const int32_t* __restrict__ tpos, int64_t T, int32_t vpr, int32_t P,
+                             float* __restrict__ ref) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < T; r += warps) {
+    const int t = __ldg(tpos + r);
+    const int j = (t >= 0 && t < P) ? t : 0;
+    const uint4* xr = x + r * vpr;
+    const uint4* wr = w_c + (int64_t)j * vpr;
+    float acc = 0.f;
+    for (int v = lane; v < vpr; v += 32) acc = dot8_bf16(__ldg(xr + v), __ldg(wr + v), acc);
+    acc = warp_sum(acc);
+    if (lane == 0) ref[r] = acc;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Row pass after the forward GEMM. With S_i = sum of the row's per-tile sums of
+// exp(z - ref_i):
+//   lse_i = ref_i + log S_i,   loss_i = lse_i - z_target = log S_i (valid rows),
+//   r_i = 1 / S_i (0 on ignored rows),  E'[i, t_i] = 1 - S_i,  x'_i = r_i x_i,
+// so that r_i E'_ij = softmax_ij - [j == t_i] (the CE gradient w.r.t. the
+// logits, "Learning Triton One Kernel at a Time: Softmax", section "Gradient")
+// and the backward is dX = (g/n) r (.) (E' W_C), dW_C = (g/n) E'^T x'.
+// A row whose S_i is not below 2^64 (E overflowed: its loss exceeds ~44 nats)
+// is listed for the exact fix-up below instead.
+// ----------------------------------------------------------------------------
+constexpr float kFixThreshold = 1.8446744e19f;  // 2^64
+
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 a, float r) {
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h)
+    o[h] = pack_bf16x2(__uint_as_float(w[h] << 16) * r, __uint_as_float(w[h] & 0xffff0000u) * r);
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void k_rows(RowArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int vpr = a.d / 8;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < a.T; r += warps) {
+    float s = 0.f;
+    for (int t = lane; t < a.tiles_n; t += 32) s += __ldg(a.rowsum + (int64_t)t * a.T + r);
+    const float S = warp_sum(s);
+    const int tp = __ldg(a.tpos + r);
+    const bool valid = tp >= 0 && tp < a.P;
+    if (!(S < kFixThreshold)) {  // overflow (or NaN): exact recomputation later
+      if (lane == 0) a.fix_list[atomicAdd(a.fix_count, 1)] = (int32_t)r;
+      continue;
+    }
+    const float rs = valid ? 1.f / S : 0.f;
+    if (lane == 0) {
+      a.lse[r] = __ldg(a.ref + r) + logf(S);
+      a.loss_rows[r] = valid ? logf(S) : 0.f;
+      a.rscale[r] = rs;
+      if (valid) a.u[r * a.ldz + tp] = (uint16_t)(pack_bf16x2(1.f - S, 0.f) & 0xffffu);
+    }
+    const uint4* xr = reinterpret_cast<const uint4*>(a.x) + r * vpr;
+    uint4* xo = reinterpret_cast<uint4*>(a.xs) + r * vpr;
+    for (int v = lane; v < vpr; v += 32) xo[v] = scale_bf16x8(__ldg(xr + v), rs);
+  }
+}
+
+// Exact recomputation of listed rows, max-shifted (section "Definition"):
+// one CTA per row recomputes the row's P logits in fp32, then rewrites lse,
+// the row loss, r_i, x'_i and the row of E' with the row max as the shift.
+constexpr int kFixThreads = 256;
+
+__device__ float block_reduce(float v, bool is_max, float* sh) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float w = __shfl_down_sync(0xffffffffu, v, o);
+    v = is_max ? fmaxf(v, w) : v + w;
+  }
+  if (lane == 0) sh[wid] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = sh[0];
+    for (int w = 1; w < kFixThreads / 32; ++w) t = is_max ? fmaxf(t, sh[w]) : t + sh[w];
+    sh[32] = t;
+  }
+  __syncthreads();
+  const float out = sh[32];
+  __syncthreads();
+  return out;
+}
+
+__device__ __forceinline__ float row_logit(const uint4* xr, const uint4* wr, int vpr) {
+  float acc = 0.f;
+  for (int v = 0; v < vpr; ++v) acc = dot8_bf16(__ldg(xr + v), __ldg(wr + v), acc);
+  return acc;
+}
+
+__global__ void __launch_bounds__(kFixThreads) k_fixup(RowArgs a) {
+  __shared__ float sh[33];
+  __shared__ float s_zt;
+  const int n = *reinterpret_cast<volatile int32_t*>(a.fix_count);
+  const int vpr = a.d / 8;
+  for (int k = blockIdx.x; k < n; k += gridDim.x) {
+    const int64_t r = a.fix_list[k];
+    const int tp = a.tpos[r];
+    const bool valid = tp >= 0 && tp < a.P;
+    const uint4* xr = reinterpret_cast<const uint4*>(a.x) + r * vpr;
+    const uint4* w = reinterpret_cast<const uint4*>(a.w_c);
+    float m = -INFINITY;
+    for (int j = threadIdx.x; j < a.P; j += kFixThreads)
+      m = fmaxf(m, row_logit(xr, w + (int64_t)j * vpr, vpr));
+    m = block_reduce(m, true, sh);
+    float sum = 0.f;
+    uint16_t* ur = a.u + r * a.ldz;
+    for (int j = threadIdx.x; j < a.P; j += kFixThreads) {
+      const float z = row_logit(xr, w + (int64_t)j * vpr, vpr);
+      const float e = expf(z - m);
+      sum += e;
+      ur[j] = valid ? (uint16_t)(pack_bf16x2(e, 0.f) & 0xffffu) : (uint16_t)0;
+      if (j == tp) s_zt = z;
+    }
+    const float S = block_reduce(sum, false, sh);  // also orders the E' writes above
+    const float rs = valid ? 1.f / S : 0.f;
+    if (threadIdx.x == 0) {
+      const float lse = m + logf(S);
+      a.lse[r] = lse;
+      a.loss_rows[r] = valid ? lse - s_zt : 0.f;
+      a.rscale[r] = rs;
+      if (valid) ur[tp] = (uint16_t)(pack_bf16x2(expf(s_zt - m) - S, 0.f) & 0xffffu);
+    }
+    uint4* xo = reinterpret_cast<uint4*>(a.xs) + r * vpr;
+    for (int v = threadIdx.x; v < vpr; v += kFixThreads) xo[v] = scale_bf16x8(__ldg(xr + v), rs);
+    __syncthreads();
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Loss: sum of the valid rows' losses over the valid-row count (Handout #16
+// CPU checks, lm_gradient), in a fixed order (deterministic).
+// ----------------------------------------------------------------------------
+__global__ void k_finalize(const float* __restrict__ loss_rows, const int32_t* __restrict__ tpos,
+                           int64_t T, int32_t P, float* __restrict__ loss,
+                           int32_t* __restrict__ n_valid) {
   __shared__ double s_sum[32], s_cnt[32];
   double s = 0.0, c = 0.0;
-  for (int b = threadIdx.x; b < nitems; b += blockDim.x) {
-    s += partials[2 * b];
-    c += partials[2 * b + 1];
+  for (int64_t i = threadIdx.x; i < T; i += blockDim.x) {
+    const int t = tpos[i];
+    if (t >= 0 && t < P) {
+      s += (double)loss_rows[i];
+      c += 1.0;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -374,9 +537,31 @@ cudaError_t launch_gather(const uint16_t* lm_head, const int32_t* cand, int32_t 
   return cudaGetLastError();
 }
 
-cudaError_t launch_finalize(const double* partials, int32_t nitems, float* loss,
-                            int32_t* n_valid, cudaStream_t s) {
-  k_finalize<<<1, 1024, 0, s>>>(partials, nitems, loss, n_valid);
+cudaError_t launch_ref_logits(const uint16_t* x, const uint16_t* w_c, const int32_t* tpos,
+                              int64_t T, int32_t d, int32_t P, float* ref, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = (int)min64((T + 7) / 8, (int64_t)num_sms() * 16);
+  k_ref_logits<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(x),
+                                      reinterpret_cast<const uint4*>(w_c), tpos, T, d / 8, P, ref);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rows(const RowArgs& a, cudaStream_t s) {
+  if (a.T == 0) return cudaSuccess;
+  const int blocks = (int)min64((a.T + 7) / 8, (int64_t)num_sms() * 16);
+  k_rows<<<blocks, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fixup(const RowArgs& a, cudaStream_t s) {
+  if (a.T == 0) return cudaSuccess;
+  k_fixup<<<num_sms(), kFixThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const float* loss_rows, const int32_t* tpos, int64_t T, int32_t P,
+                            float* loss, int32_t* n_valid, cudaStream_t s) {
+  k_finalize<<<1, 1024, 0, s>>>(loss_rows, tpos, T, P, loss, n_valid);
   return cudaGetLastError();
 }
 

@@ -153,11 +153,9 @@ constexpr int kBM = 128, kBN = 256, kBMP = 256;  // rows per CTA, cols per tile,
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-  size_t bitmap, prefix, partials, counters, w_c, z, stats, zt, total;
+  size_t bitmap, prefix, ref, rscale, loss_rows, fix_list, fix_count, w_c, u, rowsum, xs, total;
   int64_t ldz;
   int tiles_n;
-  int nitems;   // converter work items (kRowsPerItem rows each)
-  int nhalf;    // 128-row half-stripes of all pair tiles; counters = nhalf + 1 ticket
 };
 
 bool sizes_ok(int64_t T, int32_t d, int32_t V, int32_t P) {
@@ -170,27 +168,25 @@ Layout layout(int64_t T, int32_t d, int32_t V, int32_t P) {
   const size_t nw = (size_t)(V + 31) / 32;
   L.ldz = (P + 7) / 8 * 8;
   L.tiles_n = (P + kBN - 1) / kBN;
-  L.nitems = converter_items(T);
-  L.nhalf = 2 * (int)((T + kBMP - 1) / kBMP);  // both CTAs of every pair tile publish
   size_t off = 0;
-  L.bitmap = off;
-  off += align_up(nw * 4, 256);
-  L.prefix = off;
-  off += align_up(nw * 4, 256);
-  L.partials = off;
-  off += align_up((size_t)L.nitems * 16 + 16, 256);
-  L.counters = off;
-  off += align_up((size_t)(L.nhalf + 1) * 4, 256);
-  off = align_up(off, 1024);
-  L.w_c = off;
-  off += align_up((size_t)P * d * 2, 1024);
-  L.z = off;
-  off += align_up((size_t)T * L.ldz * 2, 1024);
-  L.stats = off;
-  off += align_up((size_t)L.tiles_n * T * 8, 256);
-  L.zt = off;
-  off += align_up((size_t)T * 4, 256);
-  L.total = off;
+  auto take = [&](size_t bytes, size_t align) {
+    off = align_up(off, align);
+    const size_t at = off;
+    off += bytes;
+    return at;
+  };
+  L.bitmap = take(nw * 4, 256);
+  L.prefix = take(nw * 4, 256);
+  L.ref = take((size_t)T * 4, 256);
+  L.rscale = take((size_t)T * 4, 256);
+  L.loss_rows = take((size_t)T * 4, 256);
+  L.fix_list = take((size_t)T * 4, 256);
+  L.fix_count = take(16, 256);
+  L.w_c = take((size_t)P * d * 2, 1024);
+  L.u = take((size_t)T * L.ldz * 2, 1024);
+  L.rowsum = take((size_t)L.tiles_n * T * 4, 1024);
+  L.xs = take((size_t)T * d * 2, 1024);
+  L.total = align_up(off, 1024);
   return L;
 }
 
@@ -290,21 +286,21 @@ ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t*
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint16_t* w_c = reinterpret_cast<uint16_t*>(ws + L.w_c);
-  uint16_t* z = reinterpret_cast<uint16_t*>(ws + L.z);
-  float2* stats = reinterpret_cast<float2*>(ws + L.stats);
-  float* zt = reinterpret_cast<float*>(ws + L.zt);
-  double* partials = reinterpret_cast<double*>(ws + L.partials);
-  int32_t* counters = reinterpret_cast<int32_t*>(ws + L.counters);
+  uint16_t* u = reinterpret_cast<uint16_t*>(ws + L.u);
+  float* ref = reinterpret_cast<float*>(ws + L.ref);
+  float* rowsum = reinterpret_cast<float*>(ws + L.rowsum);
+  float* loss_rows = reinterpret_cast<float*>(ws + L.loss_rows);
+  int32_t* fix_count = reinterpret_cast<int32_t*>(ws + L.fix_count);
   int32_t* kstatus = dev_status + 8;
 
-  SS_LAUNCH("gather", s,
-            launch_gather(lm_head, candidates, P, d, V, w_c, kstatus, counters, L.nhalf + 1, s));
+  SS_LAUNCH("gather", s, launch_gather(lm_head, candidates, P, d, V, w_c, kstatus, fix_count, 1, s));
   if (T > 0) {
+    SS_LAUNCH("ref_logits", s, launch_ref_logits(x, w_c, target_pos, T, d, P, ref, s));
     CUtensorMap ta, tb, tc;
     ss_status r;
     if ((r = make_map(&ta, x, d, T, d, 64, kBM)) != SS_OK) return r;
     if ((r = make_map(&tb, w_c, d, P, d, 64, kBN / 2)) != SS_OK) return r;
-    if ((r = make_map(&tc, z, P, T, L.ldz, 64, 32)) != SS_OK) return r;
+    if ((r = make_map(&tc, u, P, T, L.ldz, 64, 32)) != SS_OK) return r;
     GemmArgs a{};
     a.M = (int32_t)T;
     a.N = P;
@@ -313,35 +309,47 @@ ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t*
     a.tiles_n = L.tiles_n;
     a.num_kb = (d + 63) / 64;
     a.tpos = target_pos;
-    a.stats = stats;
-    a.zt = zt;
-    a.u = z;
-    a.ldz = L.ldz;
-    a.done = counters;
-    a.ticket = counters + L.nhalf;
-    a.lse = lse;
-    a.partials = partials;
-    a.num_items = L.nitems;
+    a.ref = ref;
+    a.rowsum = rowsum;
     a.status = kstatus;
     const int tiles = a.tiles_m * a.tiles_n;
     SS_LAUNCH("fwd_gemm_ce", s,
               launch_gemm(KIND_FWD, ta, tb, tc, a, tiles < pairs[KIND_FWD] ? tiles : pairs[KIND_FWD], s));
+    RowArgs ra{};
+    ra.rowsum = rowsum;
+    ra.ref = ref;
+    ra.tpos = target_pos;
+    ra.x = x;
+    ra.T = T;
+    ra.d = d;
+    ra.P = P;
+    ra.tiles_n = L.tiles_n;
+    ra.ldz = L.ldz;
+    ra.w_c = w_c;
+    ra.u = u;
+    ra.lse = lse;
+    ra.rscale = reinterpret_cast<float*>(ws + L.rscale);
+    ra.xs = reinterpret_cast<uint16_t*>(ws + L.xs);
+    ra.loss_rows = loss_rows;
+    ra.fix_list = reinterpret_cast<int32_t*>(ws + L.fix_list);
+    ra.fix_count = fix_count;
+    SS_LAUNCH("row_pass", s, launch_rows(ra, s));
+    SS_LAUNCH("row_fixup", s, launch_fixup(ra, s));
   }
-  SS_LAUNCH("loss_finalize", s, launch_finalize(partials, T > 0 ? L.nitems : 0, loss, n_valid, s));
+  SS_LAUNCH("loss_finalize", s, launch_finalize(loss_rows, target_pos, T, P, loss, n_valid, s));
   return SS_OK;
 }
 
-ss_status ss_ce_backward(const float* grad_loss, const ss_bf16* x, const int32_t* candidates,
-                         const int32_t* target_pos, const int32_t* vocab_pos,
-                         const int32_t* n_valid, int64_t T, int32_t d, int32_t V, int32_t P,
-                         ss_bf16* dx, ss_bf16* dW, int32_t* dev_status, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
+                         const int32_t* vocab_pos, const int32_t* n_valid, int64_t T, int32_t d,
+                         int32_t V, int32_t P, ss_bf16* dx, ss_bf16* dW, int32_t* dev_status,
+                         void* workspace, size_t workspace_bytes, void* stream) {
   if (!sizes_ok(T, d, V, P)) return SS_ERR_INVALID_ARG;
   if (grad_loss == nullptr || candidates == nullptr || vocab_pos == nullptr ||
       n_valid == nullptr || dW == nullptr || dev_status == nullptr || workspace == nullptr ||
-      (T > 0 && (x == nullptr || target_pos == nullptr || dx == nullptr)))
+      (T > 0 && dx == nullptr))
     return SS_ERR_INVALID_ARG;
-  if (!aligned16(dW) || !aligned16(workspace) || (T > 0 && (!aligned16(x) || !aligned16(dx))))
+  if (!aligned16(dW) || !aligned16(workspace) || (T > 0 && !aligned16(dx)))
     return SS_ERR_MISALIGNED;
   const Layout L = layout(T, d, V, P);
   if (workspace_bytes < L.total) return SS_ERR_WORKSPACE_TOO_SMALL;
@@ -351,7 +359,8 @@ ss_status ss_ce_backward(const float* grad_loss, const ss_bf16* x, const int32_t
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint16_t* w_c = reinterpret_cast<uint16_t*>(ws + L.w_c);
-  uint16_t* z = reinterpret_cast<uint16_t*>(ws + L.z);
+  uint16_t* u = reinterpret_cast<uint16_t*>(ws + L.u);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
   int32_t* kstatus = dev_status + 8;
 
   if (T == 0) {
@@ -360,13 +369,13 @@ ss_status ss_ce_backward(const float* grad_loss, const ss_bf16* x, const int32_t
   }
   SS_LAUNCH("zero_rows", s, launch_zero_rows(dW, V, d, vocab_pos, 0, s));
 
-  CUtensorMap ga, wb, dxs, ga2, xb;
+  CUtensorMap ua, wb, dxs, ua2, xb;
   ss_status r;
-  if ((r = make_map(&ga, z, P, T, L.ldz, 64, kBM)) != SS_OK) return r;   // U, K-major
+  if ((r = make_map(&ua, u, P, T, L.ldz, 64, kBM)) != SS_OK) return r;   // E', K-major
   if ((r = make_map(&wb, w_c, d, P, d, 64, 64)) != SS_OK) return r;      // W_C, MN-major
   if ((r = make_map(&dxs, dx, d, T, d, 64, 32)) != SS_OK) return r;      // dx store
-  if ((r = make_map(&ga2, z, P, T, L.ldz, 64, 64)) != SS_OK) return r;   // U^T, MN-major
-  if ((r = make_map(&xb, x, d, T, d, 64, 64)) != SS_OK) return r;        // x, MN-major
+  if ((r = make_map(&ua2, u, P, T, L.ldz, 64, 64)) != SS_OK) return r;   // E'^T, MN-major
+  if ((r = make_map(&xb, xs, d, T, d, 64, 64)) != SS_OK) return r;       // x', MN-major
 
   GemmArgs a{};
   a.M = (int32_t)T;
@@ -377,10 +386,11 @@ ss_status ss_ce_backward(const float* grad_loss, const ss_bf16* x, const int32_t
   a.num_kb = (P + 63) / 64;
   a.grad_loss = grad_loss;
   a.n_valid = n_valid;
+  a.rscale = reinterpret_cast<const float*>(ws + L.rscale);
   a.status = kstatus;
   int tiles = a.tiles_m * a.tiles_n;
   SS_LAUNCH("dx_gemm", s,
-            launch_gemm(KIND_DX, ga, wb, dxs, a, tiles < pairs[KIND_DX] ? tiles : pairs[KIND_DX], s));
+            launch_gemm(KIND_DX, ua, wb, dxs, a, tiles < pairs[KIND_DX] ? tiles : pairs[KIND_DX], s));
 
   GemmArgs b{};
   b.M = P;
@@ -397,7 +407,7 @@ ss_status ss_ce_backward(const float* grad_loss, const ss_bf16* x, const int32_t
   b.status = kstatus;
   tiles = b.tiles_m * b.tiles_n;
   SS_LAUNCH("dw_gemm_scatter", s,
-            launch_gemm(KIND_DW, ga2, xb, ga2, b, tiles < pairs[KIND_DW] ? tiles : pairs[KIND_DW], s));
+            launch_gemm(KIND_DW, ua2, xb, ua2, b, tiles < pairs[KIND_DW] ? tiles : pairs[KIND_DW], s));
   return SS_OK;
 }
 

@@ -15,21 +15,14 @@ struct GemmArgs {
   int32_t M, N, K;           // output rows, output cols, contraction length
   int32_t tiles_m, tiles_n;  // ceil(M / 256) (CTA-pair rows), ceil(N / 256)
   int32_t num_kb;            // ceil(K / 64)
-  // forward epilogue
+  // forward epilogue: E = exp(z - ref) and its per-tile row sums
   const int32_t* tpos;  // [M] target position of each row, -1 = ignored
-  float2* stats;        // [tiles_n][M] per-tile (row max, sum of exp(z - max))
-  float* zt;            // [M] fp32 logit of the target column
-  // forward converter warps: logits -> softmax - onehot, in place
-  uint16_t* u;          // [M][ldz] bf16 logits, rewritten as softmax - onehot
-  int64_t ldz;
-  int32_t* done;        // [ceil(M / 128)] finished tiles per 128-row half-stripe
-  int32_t* ticket;      // converter work-item counter
-  float* lse;           // [M]
-  double* partials;     // [2 * num_items] per work item: (sum of row losses, valid rows)
-  int32_t num_items;    // ceil(M / kRowsPerItem)
-  // dX / dW epilogue scale g / n
+  const float* ref;     // [M] reference logit of each row
+  float* rowsum;        // [tiles_n][M] sum over each 256-column tile of exp(z - ref)
+  // dX / dW epilogue scale g / n (dX also times rscale[row])
   const float* grad_loss;
   const int32_t* n_valid;
+  const float* rscale;  // [M] (dX) 1 / S_i, 0 on ignored rows
   // dW epilogue
   const int32_t* cand;  // [M] class id of each output row
   uint16_t* dW;         // [V][N] bf16
@@ -37,15 +30,12 @@ struct GemmArgs {
   int32_t* status;  // dev_status + 8 (error word, detail word)
 };
 
-constexpr int kRowsPerItem = 4;  // rows one converter warp takes at a time
-
 enum GemmKind { KIND_FWD = 0, KIND_DX = 1, KIND_DW = 2 };
 
 // Launches `pairs` CTA pairs (clusters of 2) of the persistent GEMM kernel.
 cudaError_t launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& c, const GemmArgs& args, int pairs, cudaStream_t s);
 int gemm_smem_bytes();
-int gemm_rows_per_tile();
 const void* gemm_kernel_ptr(int kind);
 int gemm_max_pairs(int kind, int sms);
 
@@ -60,11 +50,32 @@ cudaError_t launch_build_emit(const int32_t* targets, int64_t T, int32_t V, int3
 cudaError_t launch_gather(const uint16_t* lm_head, const int32_t* cand, int32_t P, int32_t d,
                           int32_t V, uint16_t* w_c, int32_t* status, int32_t* zero_words,
                           int32_t n_zero_words, cudaStream_t s);
-cudaError_t launch_finalize(const double* partials, int32_t nitems, float* loss,
-                            int32_t* n_valid, cudaStream_t s);
+// ref[i] = x_i . W_C[target_pos_i] (W_C[0] on ignored rows), fp32.
+cudaError_t launch_ref_logits(const uint16_t* x, const uint16_t* w_c, const int32_t* tpos,
+                              int64_t T, int32_t d, int32_t P, float* ref, cudaStream_t s);
+// Row pass after the forward GEMM (see ce_kernels.cu).
+struct RowArgs {
+  const float* rowsum;  // [tiles_n][T]
+  const float* ref;     // [T]
+  const int32_t* tpos;  // [T]
+  const uint16_t* x;    // [T][d]
+  int64_t T;
+  int32_t d, P, tiles_n;
+  int64_t ldz;
+  const uint16_t* w_c;  // [P][d] (fix-up)
+  uint16_t* u;          // [T][ldz] E, patched at the target column
+  float* lse;           // [T]
+  float* rscale;        // [T]
+  uint16_t* xs;         // [T][d] x' = rscale * x
+  float* loss_rows;     // [T]
+  int32_t* fix_list;    // [T] rows whose E overflowed
+  int32_t* fix_count;   // [1]
+};
+cudaError_t launch_rows(const RowArgs& a, cudaStream_t s);
+cudaError_t launch_fixup(const RowArgs& a, cudaStream_t s);
+cudaError_t launch_finalize(const float* loss_rows, const int32_t* tpos, int64_t T, int32_t P,
+                            float* loss, int32_t* n_valid, cudaStream_t s);
 cudaError_t launch_zero_rows(uint16_t* dW, int32_t V, int32_t d, const int32_t* vocab_pos,
                              int all_rows, cudaStream_t s);
-
-inline int converter_items(int64_t T) { return (int)((T + kRowsPerItem - 1) / kRowsPerItem); }
 
 }  // namespace ssb

@@ -170,6 +170,55 @@ def test_uniform_logits_give_log_p():
     assert np.max(np.abs(g["lse"] - np.log(P))) <= 1e-5
 
 
+def test_rows_with_huge_loss_are_recomputed_exactly():
+    """Rows whose target logit lies ~120 below another candidate's.
+
+    The forward stores exp(z - z_target); such rows overflow it and take the
+    exact recomputation path. lse, loss and gradients must still match the
+    oracle, on those rows and on the rest.
+    """
+    T, d, V, P, seed = 300, 64, 1000, 384, 21
+    x, lm, t = random_case(T, d, V, P, seed)
+    xf = wl.bits_to_f32(x).copy()
+    lmf = wl.bits_to_f32(lm)
+    rng = np.random.default_rng(seed)
+    cand, _, _, _ = oc.build_candidates(t, V, P, 0)
+    for i in (3, 77, 150):                 # valid rows: push another class far above the target
+        a = int(cand[(np.searchsorted(cand, t[i]) + 5) % P]) if t[i] >= 0 else int(cand[5])
+        if t[i] < 0:
+            t[i] = int(cand[0])
+        diff = lmf[a] - lmf[t[i]]
+        xf[i] = 60.0 * diff / (diff @ diff)
+    t[200] = -1                             # an ignored row far from its reference class
+    diff = lmf[int(cand[7])] - lmf[int(cand[0])]
+    xf[200] = 60.0 * diff / (diff @ diff)
+    x = wl.bf16_bits(xf)
+    assert np.unique(t[t >= 0]).size <= P
+    g = run_path(x, lm, t, P, 0)
+    o = oracle_run(x, lm, t, P, 0)
+    assert np.all(np.isfinite(g["lse"]))
+    assert max(o["loss_rows"][[3, 77, 150]]) > 50      # the rows really are extreme
+    compare_full(g, o, t)
+    np.testing.assert_allclose(g["lse"][[3, 77, 150, 200]], o["lse"][[3, 77, 150, 200]], atol=LSE_ATOL)
+
+
+def test_backward_can_be_repeated():
+    x, lm, t = random_case(700, 128, 3001, 1024, 22)
+    T, d, V, P = 700, 128, 3001, 1024
+    ce = capi.SampledCE(T, d, V, P)
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    lt = torch.from_numpy(lm.view(np.int16)).view(torch.bfloat16).cuda()
+    ce.build(torch.from_numpy(t).cuda(), 5)
+    ce.forward(xt, lt)
+    ce.backward()
+    dx1, dw1 = ce.dx.clone(), ce.dW.clone()
+    ce.grad_loss.fill_(2.0)
+    ce.backward()
+    torch.cuda.synchronize()
+    assert torch.equal(ce.dx.float(), (2 * dx1.float()).bfloat16().float())
+    assert torch.equal(ce.dW.float(), (2 * dw1.float()).bfloat16().float())
+
+
 def test_deterministic():
     x, lm, t = random_case(1000, 200, 5003, 3000, 13)
     a = run_path(x, lm, t, 3000, 17)
@@ -190,8 +239,8 @@ def test_kernel_timing_records_every_kernel():
         capi.ss_timing_enable(False)
     rec = capi.ss_timing_read()
     capi.ss_timing_reset()
-    for k in ("build_mark", "build_emit", "gather", "fwd_gemm_ce", "loss_finalize", "zero_rows",
-              "dx_gemm", "dw_gemm_scatter"):
+    for k in ("build_mark", "build_emit", "gather", "ref_logits", "fwd_gemm_ce", "row_pass",
+              "row_fixup", "loss_finalize", "zero_rows", "dx_gemm", "dw_gemm_scatter"):
         assert rec[k][0] == 1 and rec[k][1] > 0, (k, rec)
 
 
