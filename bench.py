@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=wl.HEADLINE, choices=list(wl.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload with this many tokens instead (profiling a smaller case)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256,
@@ -419,6 +421,9 @@ def run_ours(args, w):
 def main():
     args = parse()
     w = wl.WORKLOADS[args.workload]
+    if args.tokens:
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}[T={args.tokens}]", T=args.tokens)
     if args.impl == "reference":
         run_reference(args, w)
     else:
