@@ -29,9 +29,11 @@
 // and its 128-column half of B; the pair's leader issues M=256, N=256, K=16
 // MMAs that read both CTAs' shared memory and write 128 rows x 256 fp32
 // columns into each CTA's TMEM. Per CTA, 192 threads, persistent over tiles:
-//   warp 0      TMA producer, 6-stage ring of 32 KB (A 128x64 + B 128x64)
+//   warp 0      TMA producer, ring of 32 KB stages (A 128x64 + B 128x64):
+//               6 in the forward, 7 in dX and dW
 //   warp 1      TMEM owner (2 x 256 columns); in the leader, the MMA issuer
-//   warps 2..5  epilogue: TMEM -> registers -> math -> shared -> TMA store
+//   warps 2..5  epilogue: TMEM -> registers -> math -> global (forward: through a
+//               swizzled shared-memory box and TMA stores; dX, dW: 16-byte stores)
 // Two TMEM accumulators let the epilogue of tile i overlap the MMAs of i+1.
 #include "sm100.cuh"
 #include "ss_internal.h"
@@ -41,34 +43,42 @@ namespace ssb {
 constexpr int BM = 128;          // rows per CTA (256 per pair)
 constexpr int BN = 256;          // output columns per tile
 constexpr int BNH = BN / 2;      // B columns held by each CTA of the pair
-constexpr int BK = 64, STAGES = 6;
+constexpr int BK = 64;
 constexpr int A_STAGE = BM * BK * 2;   // 16 KB
 constexpr int B_STAGE = BNH * BK * 2;  // 16 KB
 constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
 constexpr int EPI_BUF = 32 * 64 * 2;  // one 32-row x 64-column bf16 box (4 KB)
 constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int NUM_THREADS = 192;
 constexpr float LOG2E = 1.4426950408889634f;
 
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-
+// Stages: as many as shared memory allows. The forward's E is a 2.4 GB write
+// stream, which TMA bulk stores from a staging box handle far better than
+// 16-byte stores from registers (1.47 vs 1.89 ms measured); the box costs
+// one stage. dX and dW store little and use the 7th stage instead.
 template <int KIND>
 struct Op;
 template <>
 struct Op<KIND_FWD> {  // A = x (K-major), B = W_C (K-major)
-  static constexpr int A_MN = 0, B_MN = 0;
+  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6;
 };
 template <>
 struct Op<KIND_DX> {  // A = E' (K-major), B = W_C viewed [K=P][N=d] (MN-major)
-  static constexpr int A_MN = 0, B_MN = 1;
+  static constexpr int A_MN = 0, B_MN = 1, TMA_STORE = 0, STAGES = 7;
 };
 template <>
 struct Op<KIND_DW> {  // A = E' viewed [K=T][M=P] (MN-major), B = x' viewed [K=T][N=d] (MN-major)
-  static constexpr int A_MN = 1, B_MN = 1;
+  static constexpr int A_MN = 1, B_MN = 1, TMA_STORE = 0, STAGES = 7;
 };
+template <int KIND>
+constexpr int smem_bytes() {
+  return 1024 + Op<KIND>::STAGES * STAGE_BYTES + (Op<KIND>::TMA_STORE ? EPI_BYTES : 0) + BAR_BYTES;
+}
+static_assert(smem_bytes<KIND_FWD>() <= 232448 && smem_bytes<KIND_DX>() <= 232448 &&
+                  smem_bytes<KIND_DW>() <= 232448,
+              "shared memory budget");
 
 SS_DEV void raise_abort(volatile int* abort_flag, int32_t* status, int kind) {
   *abort_flag = 1;
@@ -93,8 +103,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
+  constexpr int STAGES = Op<KIND>::STAGES;
   uint8_t* epi_smem = smem + STAGES * STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + EPI_BYTES);
+  uint64_t* full =
+      reinterpret_cast<uint64_t*>(epi_smem + (Op<KIND>::TMA_STORE ? EPI_BYTES : 0));
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -133,6 +145,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&tma_a);
       tma_prefetch_desc(&tma_b);
     }
+    // B (W_C, or x' in dW) is reused by every tile: keep it in L2
+    const uint64_t keep_b = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -157,10 +171,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tma_load_2d_pair(sa, &tma_a, bar, k0, m0);
           }
           if (Op<KIND>::B_MN) {
-            tma_load_2d_pair(sb, &tma_b, bar, nh0, k0);
-            tma_load_2d_pair(sb + 8192, &tma_b, bar, nh0 + 64, k0);
+            tma_load_2d_pair_hint(sb, &tma_b, bar, nh0, k0, keep_b);
+            tma_load_2d_pair_hint(sb + 8192, &tma_b, bar, nh0 + 64, k0, keep_b);
           } else {
-            tma_load_2d_pair(sb, &tma_b, bar, k0, nh0);
+            tma_load_2d_pair_hint(sb, &tma_b, bar, k0, nh0, keep_b);
           }
         }
         __syncwarp();
@@ -229,6 +243,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const int e = warp - 2;   // staging slot
     int it = 0;
     uint32_t store_ctr = 0;
+    // the forward's E is a write-once stream larger than L2: evict it first
+    const uint64_t store_policy = KIND == KIND_FWD ? policy_evict_first() : 0;
     float scale = 1.f;  // dX / dW: g / n (0 when no row is valid)
     if (KIND != KIND_FWD) {
       const int nv = __ldg(args.n_valid);
@@ -312,7 +328,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           for (int j = 0; j < 64; ++j) v[j] *= scale;
         }
 
-        if (KIND == KIND_FWD || KIND == KIND_DX) {
+        if (Op<KIND>::TMA_STORE) {
           // bf16 tile -> swizzled staging box -> TMA store
           uint8_t* buf = epi_smem + (e * 2 + (store_ctr & 1)) * EPI_BUF;
           if (lane == 0) bulk_wait_read<1>();
@@ -328,10 +344,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           fence_async_smem();
           __syncwarp();
           if (lane == 0 && m0 + q * 32 < args.M) {
-            tma_store_2d(&tma_c, buf, col0, m0 + q * 32);
+            if (KIND == KIND_FWD)
+              tma_store_2d_hint(&tma_c, buf, col0, m0 + q * 32, store_policy);
+            else
+              tma_store_2d(&tma_c, buf, col0, m0 + q * 32);
             bulk_commit();
           }
           ++store_ctr;
+        } else if (KIND != KIND_DW) {
+          // bf16 row segment straight from registers (16-byte stores)
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(args.out + (size_t)row * args.ld_out + col0);
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+              if (col0 + cc * 8 < args.N) {
+                const uint4 w = make_uint4(pack_bf16x2(v[cc * 8 + 0], v[cc * 8 + 1]),
+                                           pack_bf16x2(v[cc * 8 + 2], v[cc * 8 + 3]),
+                                           pack_bf16x2(v[cc * 8 + 4], v[cc * 8 + 5]),
+                                           pack_bf16x2(v[cc * 8 + 6], v[cc * 8 + 7]));
+                if (KIND == KIND_FWD)
+                  __stcs(dst + cc, w);  // E is a write-once stream: do not keep it in L2
+                else
+                  dst[cc] = w;
+              }
+            }
+          }
         } else {  // KIND_DW: row `row` of dW_C goes to row cand[row] of dW
           if (row_ok && cls >= 0 && cls < args.V) {
             uint4* dst = reinterpret_cast<uint4*>(args.dW + (size_t)cls * args.N + col0);
@@ -373,7 +410,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-int gemm_smem_bytes() { return SMEM_BYTES; }
+int gemm_smem_bytes(int kind) {
+  switch (kind) {
+    case KIND_FWD: return smem_bytes<KIND_FWD>();
+    case KIND_DX: return smem_bytes<KIND_DX>();
+    default: return smem_bytes<KIND_DW>();
+  }
+}
 
 const void* gemm_kernel_ptr(int kind) {
   switch (kind) {
@@ -388,7 +431,7 @@ int gemm_max_pairs(int kind, int sms) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (sms / 2));
   cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.dynamicSmemBytes = gemm_smem_bytes(kind);
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
   attr.val.clusterDim.x = 2;
@@ -408,9 +451,9 @@ cudaError_t launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b, co
                         const GemmArgs& args, int pairs, cudaStream_t s) {
   dim3 g(2 * pairs), blk(NUM_THREADS);
   switch (kind) {
-    case KIND_FWD: k_gemm<KIND_FWD><<<g, blk, SMEM_BYTES, s>>>(a, b, c, args); break;
-    case KIND_DX: k_gemm<KIND_DX><<<g, blk, SMEM_BYTES, s>>>(a, b, c, args); break;
-    default: k_gemm<KIND_DW><<<g, blk, SMEM_BYTES, s>>>(a, b, c, args); break;
+    case KIND_FWD: k_gemm<KIND_FWD><<<g, blk, smem_bytes<KIND_FWD>(), s>>>(a, b, c, args); break;
+    case KIND_DX: k_gemm<KIND_DX><<<g, blk, smem_bytes<KIND_DX>(), s>>>(a, b, c, args); break;
+    default: k_gemm<KIND_DW><<<g, blk, smem_bytes<KIND_DW>(), s>>>(a, b, c, args); break;
   }
   return cudaGetLastError();
 }

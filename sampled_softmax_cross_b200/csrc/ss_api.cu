@@ -55,7 +55,7 @@ ss_status ensure_device(int* sms, int* max_pairs = nullptr) {
       for (int k = 0; k < 3; ++k) {
         SS_CUDA(cudaFuncSetAttribute(gemm_kernel_ptr(k),
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     gemm_smem_bytes()),
+                                     gemm_smem_bytes(k)),
                 "cudaFuncSetAttribute");
         d.max_pairs[k] = gemm_max_pairs(k, d.sms);
       }
@@ -311,6 +311,8 @@ ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t*
     a.tpos = target_pos;
     a.ref = ref;
     a.rowsum = rowsum;
+    a.out = u;
+    a.ld_out = L.ldz;
     a.status = kstatus;
     const int tiles = a.tiles_m * a.tiles_n;
     SS_LAUNCH("fwd_gemm_ce", s,
@@ -387,6 +389,8 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   a.grad_loss = grad_loss;
   a.n_valid = n_valid;
   a.rscale = reinterpret_cast<const float*>(ws + L.rscale);
+  a.out = dx;
+  a.ld_out = d;
   a.status = kstatus;
   int tiles = a.tiles_m * a.tiles_n;
   SS_LAUNCH("dx_gemm", s,

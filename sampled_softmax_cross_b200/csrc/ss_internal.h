@@ -23,6 +23,9 @@ struct GemmArgs {
   const float* grad_loss;
   const int32_t* n_valid;
   const float* rscale;  // [M] (dX) 1 / S_i, 0 on ignored rows
+  // forward / dX epilogue without TMA store: output rows
+  uint16_t* out;        // [M][ld_out] bf16 (E for the forward, dx for dX)
+  int64_t ld_out;
   // dW epilogue
   const int32_t* cand;  // [M] class id of each output row
   uint16_t* dW;         // [V][N] bf16
@@ -35,7 +38,7 @@ enum GemmKind { KIND_FWD = 0, KIND_DX = 1, KIND_DW = 2 };
 // Launches `pairs` CTA pairs (clusters of 2) of the persistent GEMM kernel.
 cudaError_t launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& c, const GemmArgs& args, int pairs, cudaStream_t s);
-int gemm_smem_bytes();
+int gemm_smem_bytes(int kind);
 const void* gemm_kernel_ptr(int kind);
 int gemm_max_pairs(int kind, int sms);
 
