@@ -78,18 +78,29 @@ __global__ void __launch_bounds__(kBuildThreads)
   {
     const int64_t n4 = T >> 2;
     const int4* t4 = reinterpret_cast<const int4*>(targets);
-    for (int64_t i = tid; i < n4; i += kBuildThreads) {
-      const int4 q = __ldg(t4 + i);
-      const int tv[4] = {q.x, q.y, q.z, q.w};
+    // 8 vector loads in flight per thread before the shared-memory atomics
+    for (int64_t i0 = tid; i0 < n4; i0 += 8 * kBuildThreads) {
+      int4 q[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = tv[j];
-        if (t == -1) continue;
-        if (t < -1 || t >= V) {
-          atomicMin(&s_bad, (int)min64(4 * i + j, INT_MAX));
-          continue;
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + (int64_t)u * kBuildThreads;
+        q[u] = i < n4 ? __ldg(t4 + i) : make_int4(-1, -1, -1, -1);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + (int64_t)u * kBuildThreads;
+        const int tv[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = tv[j];
+          if (t == -1) continue;
+          if (t < -1 || t >= V) {
+            atomicMin(&s_bad, (int)min64(4 * i + j, INT_MAX));
+            continue;
+          }
+          const uint32_t bit = 1u << (t & 31);
+          if (!(bm[t >> 5] & bit)) atomicOr(&bm[t >> 5], bit);  // frequent classes: mostly set already
         }
-        atomicOr(&bm[t >> 5], 1u << (t & 31));
       }
     }
     for (int64_t i = 4 * n4 + tid; i < T; i += kBuildThreads) {
@@ -303,16 +314,35 @@ __global__ void k_ref_logits(const uint4* __restrict__ x, const uint4* __restric
                              const int32_t* __restrict__ tpos, int64_t T, int32_t vpr, int32_t P,
                              float* __restrict__ ref) {
   const int lane = threadIdx.x & 31;
+  const int64_t pairs = (T + 1) / 2;  // two rows per warp iteration, all loads in flight
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < T; r += warps) {
-    const int t = __ldg(tpos + r);
-    const int j = (t >= 0 && t < P) ? t : 0;
-    const uint4* xr = x + r * vpr;
-    const uint4* wr = w_c + (int64_t)j * vpr;
-    float acc = 0.f;
-    for (int v = lane; v < vpr; v += 32) acc = dot8_bf16(__ldg(xr + v), __ldg(wr + v), acc);
-    acc = warp_sum(acc);
-    if (lane == 0) ref[r] = acc;
+  for (int64_t pi = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); pi < pairs; pi += warps) {
+    float acc[2] = {0.f, 0.f};
+    for (int v0 = 0; v0 < vpr; v0 += 96) {
+      uint4 xa[2][3], wa[2][3];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int64_t r = 2 * pi + k;
+        const int t = r < T ? __ldg(tpos + r) : -1;
+        const int j = (t >= 0 && t < P) ? t : 0;
+#pragma unroll
+        for (int h = 0; h < 3; ++h) {
+          const int v = v0 + lane + 32 * h;
+          const bool ok = r < T && v < vpr;
+          xa[k][h] = ok ? __ldg(x + r * vpr + v) : make_uint4(0, 0, 0, 0);
+          wa[k][h] = ok ? __ldg(w_c + (int64_t)j * vpr + v) : make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int h = 0; h < 3; ++h) acc[k] = dot8_bf16(xa[k][h], wa[k][h], acc[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float sum = warp_sum(acc[k]);
+      if (lane == 0 && 2 * pi + k < T) ref[2 * pi + k] = sum;
+    }
   }
 }
 
@@ -338,30 +368,69 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 a, float r) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// Each warp takes 8 consecutive rows. For the tile sums (stored tile-major)
+// lane l adds tiles (l / 8), (l / 8) + 4, ... of row (l % 8), so every load
+// instruction reads whole 32-byte sectors; the four partial sums of a row are
+// then combined in a fixed order. The x' rows are written 4 at a time with
+// all their loads in flight.
+constexpr int kRowsPerWarp = 8;
+
 __global__ void k_rows(RowArgs a) {
   const int lane = threadIdx.x & 31;
   const int vpr = a.d / 8;
+  const int64_t groups = (a.T + kRowsPerWarp - 1) / kRowsPerWarp;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < a.T; r += warps) {
+  for (int64_t gidx = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); gidx < groups;
+       gidx += warps) {
+    const int64_t r = gidx * kRowsPerWarp + (lane & 7);
+    const bool in = r < a.T;
     float s = 0.f;
-    for (int t = lane; t < a.tiles_n; t += 32) s += __ldg(a.rowsum + (int64_t)t * a.T + r);
-    const float S = warp_sum(s);
-    const int tp = __ldg(a.tpos + r);
+    if (in)
+      for (int t = lane >> 3; t < a.tiles_n; t += 4) s += __ldg(a.rowsum + (int64_t)t * a.T + r);
+    s += __shfl_xor_sync(0xffffffffu, s, 8);
+    s += __shfl_xor_sync(0xffffffffu, s, 16);
+    const float S = s;  // identical in the four lanes of the row
+    const int tp = in ? __ldg(a.tpos + r) : -1;
     const bool valid = tp >= 0 && tp < a.P;
-    if (!(S < kFixThreshold)) {  // overflow (or NaN): exact recomputation later
-      if (lane == 0) a.fix_list[atomicAdd(a.fix_count, 1)] = (int32_t)r;
-      continue;
+    const bool fix = in && !(S < kFixThreshold);  // overflow (or NaN): exact recomputation later
+    const float rs = (in && valid && !fix) ? 1.f / S : 0.f;
+    if (lane < 8) {
+      if (in && fix) a.fix_list[atomicAdd(a.fix_count, 1)] = (int32_t)r;
+      if (in && !fix) {
+        a.lse[r] = __ldg(a.ref + r) + logf(S);
+        a.loss_rows[r] = valid ? logf(S) : 0.f;
+        a.rscale[r] = rs;
+        if (valid) a.u[r * a.ldz + tp] = (uint16_t)(pack_bf16x2(1.f - S, 0.f) & 0xffffu);
+      }
     }
-    const float rs = valid ? 1.f / S : 0.f;
-    if (lane == 0) {
-      a.lse[r] = __ldg(a.ref + r) + logf(S);
-      a.loss_rows[r] = valid ? logf(S) : 0.f;
-      a.rscale[r] = rs;
-      if (valid) a.u[r * a.ldz + tp] = (uint16_t)(pack_bf16x2(1.f - S, 0.f) & 0xffffu);
+    const unsigned todo = __ballot_sync(0xffffffffu, lane < 8 && in && !fix);
+    for (int k0 = 0; k0 < kRowsPerWarp; k0 += 4) {
+      uint4 in_v[4][3];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int64_t rr = gidx * kRowsPerWarp + k0 + k;
+        const uint4* xr = reinterpret_cast<const uint4*>(a.x) + rr * vpr;
+#pragma unroll
+        for (int h = 0; h < 3; ++h) {
+          const int v = lane + 32 * h;
+          if (((todo >> (k0 + k)) & 1u) && v < vpr) in_v[k][h] = __ldg(xr + v);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (!((todo >> (k0 + k)) & 1u)) continue;
+        const float rk = __shfl_sync(0xffffffffu, rs, k0 + k);
+        const int64_t rr = gidx * kRowsPerWarp + k0 + k;
+        const uint4* xr = reinterpret_cast<const uint4*>(a.x) + rr * vpr;
+        uint4* xo = reinterpret_cast<uint4*>(a.xs) + rr * vpr;
+#pragma unroll
+        for (int h = 0; h < 3; ++h) {
+          const int v = lane + 32 * h;
+          if (v < vpr) xo[v] = scale_bf16x8(in_v[k][h], rk);
+        }
+        for (int v = lane + 96; v < vpr; v += 32) xo[v] = scale_bf16x8(__ldg(xr + v), rk);
+      }
     }
-    const uint4* xr = reinterpret_cast<const uint4*>(a.x) + r * vpr;
-    uint4* xo = reinterpret_cast<uint4*>(a.xs) + r * vpr;
-    for (int v = lane; v < vpr; v += 32) xo[v] = scale_bf16x8(__ldg(xr + v), rs);
   }
 }
 
@@ -444,7 +513,23 @@ __global__ void k_finalize(const float* __restrict__ loss_rows, const int32_t* _
                            int32_t* __restrict__ n_valid) {
   __shared__ double s_sum[32], s_cnt[32];
   double s = 0.0, c = 0.0;
-  for (int64_t i = threadIdx.x; i < T; i += blockDim.x) {
+  // each thread takes runs of 4 consecutive rows (T rounded down to a multiple
+  // of 4 here; the rest below), fixed order
+  const int64_t T4 = T & ~int64_t(3);
+  for (int64_t i = 4 * (int64_t)threadIdx.x; i < T4; i += 4 * (int64_t)blockDim.x) {
+    const float4 l = __ldg(reinterpret_cast<const float4*>(loss_rows + i));
+    const int4 t = __ldg(reinterpret_cast<const int4*>(tpos + i));
+    const float lv[4] = {l.x, l.y, l.z, l.w};
+    const int tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (tv[u] >= 0 && tv[u] < P) {
+        s += (double)lv[u];
+        c += 1.0;
+      }
+    }
+  }
+  for (int64_t i = T4 + threadIdx.x; i < T; i += blockDim.x) {
     const int t = tpos[i];
     if (t >= 0 && t < P) {
       s += (double)loss_rows[i];
@@ -540,7 +625,7 @@ cudaError_t launch_gather(const uint16_t* lm_head, const int32_t* cand, int32_t 
 cudaError_t launch_ref_logits(const uint16_t* x, const uint16_t* w_c, const int32_t* tpos,
                               int64_t T, int32_t d, int32_t P, float* ref, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  const int blocks = (int)min64((T + 7) / 8, (int64_t)num_sms() * 16);
+  const int blocks = (int)min64(((T + 1) / 2 + 7) / 8, (int64_t)num_sms() * 16);
   k_ref_logits<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(x),
                                       reinterpret_cast<const uint4*>(w_c), tpos, T, d / 8, P, ref);
   return cudaGetLastError();
@@ -548,14 +633,17 @@ cudaError_t launch_ref_logits(const uint16_t* x, const uint16_t* w_c, const int3
 
 cudaError_t launch_rows(const RowArgs& a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  const int blocks = (int)min64((a.T + 7) / 8, (int64_t)num_sms() * 16);
+  const int64_t groups = (a.T + kRowsPerWarp - 1) / kRowsPerWarp;  // per warp; 8 warps per block
+  const int blocks = (int)min64((groups + 7) / 8, (int64_t)num_sms() * 16);
   k_rows<<<blocks, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fixup(const RowArgs& a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  k_fixup<<<num_sms(), kFixThreads, 0, s>>>(a);
+  // Rows are flagged only when their loss is enormous, so one CTA (which
+  // finds the list empty in the common case) is enough.
+  k_fixup<<<1, kFixThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
