@@ -39,7 +39,7 @@ METRIC = "tokens/s fused sampled-CE fwd+bwd at P=24576,d=768; % of BF16 tensor p
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=wl.HEADLINE, choices=list(wl.WORKLOADS))
@@ -108,8 +108,9 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.thread.join(timeout=5)
-        # samples taken while the timed region ran (the first one marks its start)
-        lines = self.lines[max(0, self.n_before - 1):]
+        # samples taken while the timed region ran (if it was shorter than
+        # one interval, the last sample before it)
+        lines = self.lines[self.n_before:] or self.lines[max(0, self.n_before - 1):]
         rows = [r for r in csv.reader(io.StringIO("".join(lines))) if len(r) >= 9]
         if not rows:
             return None

@@ -35,7 +35,8 @@
  *   [6] first token index with a bad target, else -1
  *   [7] number of classes marked (P when the build succeeded)
  *   [8] forward/backward kernel error (ss_status, 0 = none)
- *   [9] detail for [8] (kernel id)      [10..15] reserved (0)
+ *   [9] detail for [8] (kernel id)      [10..11] written by
+ *   ss_selftest_wait_limit only          [12..15] reserved (0)
  */
 #ifndef SAMPLED_CE_H
 #define SAMPLED_CE_H
@@ -181,6 +182,40 @@ SS_API const char* ss_last_cuda_error(void);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 SS_API int32_t ss_version(void);
+
+/* Positions in C of each token's prefix target (sampled_softmax.py: module
+ * docstring, CandidateBuilder.build and the SampledLoss field prefix_pos).
+ * For token i with a valid target t_i the prefix target is
+ * p_i = prefix_table[t_i]; prefix_pos[i] = vocab_pos[p_i] when p_i is a class
+ * of C, and -1 otherwise: when p_i is a class outside C (the prefix target is
+ * dropped for that token, so prefix targets never add classes to C), when
+ * p_i = -1 ("no prefix"), and for an ignored token (t_i = -1). The caller's
+ * loss reads -1 as a no-op.
+ * In:  prefix_table [V] int32, entries in [-1, V); targets [T] and vocab_pos
+ *      [V] of the same microbatch as given to / written by ss_build_candidates.
+ * Out: prefix_pos [T] int32.
+ * A table entry outside [-1, V) or a target outside [-1, V) gives -1 for that
+ * token and sets dev_status[8] = SS_ERR_BAD_INDEX (first error wins) with
+ * dev_status[9] = 2 (table entry) or 3 (target). Needs no workspace. */
+SS_API ss_status ss_prefix_positions(const int32_t* prefix_table, const int32_t* targets,
+                                     const int32_t* vocab_pos, int64_t T, int32_t V,
+                                     int32_t* prefix_pos, int32_t* dev_status, void* stream);
+
+/* Self-test of the failure path every pipeline wait in the kernels shares
+ * (the pages have no counterpart). Each wait on a TMA / MMA barrier is
+ * bounded: after 2 s without progress the waiting warp raises its CTA's abort
+ * flag, records SS_ERR_KERNEL_TIMEOUT in dev_status[8] (first error wins,
+ * detail in [9]) and its kernel returns, so a stalled pipeline leaves an
+ * error status and a usable context instead of a hung GPU. This call
+ * launches one CTA whose first warp waits on a barrier that nothing
+ * completes; its second warp starts a like wait 0.25 s later and must leave
+ * through the abort flag. Afterwards, once the stream reaches it (about 2 s):
+ *   dev_status[8]  = SS_ERR_KERNEL_TIMEOUT if [8] was 0 before
+ *   dev_status[9]  = 107 (the self-test's kernel id)
+ *   dev_status[10] = 1 if the second warp left through the abort flag
+ *   dev_status[11] = the first warp's wait in whole milliseconds
+ * Returns SS_OK once the kernel is enqueued. Occupies one SM for ~2 s. */
+SS_API ss_status ss_selftest_wait_limit(int32_t* dev_status, void* stream);
 
 /* Kernel timing for diagnostics. While enabled, each kernel launch the library
  * makes is bracketed by two CUDA events recorded on its stream (a pool of

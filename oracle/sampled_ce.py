@@ -146,6 +146,42 @@ def build_candidates(targets: np.ndarray, V: int, P: int, offset: int = 0,
     return candidates, target_pos, vocab_pos, info
 
 
+def prefix_positions(prefix_table: np.ndarray, targets: np.ndarray,
+                     vocab_pos: np.ndarray) -> np.ndarray:
+    """Position in C of each token's prefix target (CandidateBuilder.build, and
+    the SampledLoss field ``prefix_pos``; module docstring: a prefix target not
+    in C is dropped for that token, so it never forces a class into C).
+
+    Steps, in the page's order:
+      1. prefix target of token i = prefix_table[targets[i]];
+      2. its position = vocab_pos[prefix target], where the class map gives -1
+         for classes outside C and for the "no prefix" marker -1 (the page
+         keeps a sentinel entry at index V that stays -1 for this).
+
+    Reading: an ignored token (target -1) has no prefix target, so its
+    position is -1 (the page's ``np.take`` would wrap -1 to the table's last
+    entry; the kernel reads -1 targets as no-ops either way). Table entries
+    and targets outside [-1, V) are rejected.
+
+    Returns prefix_pos int64 [T].
+    """
+    prefix_table = np.asarray(prefix_table, dtype=np.int64)
+    targets = np.asarray(targets, dtype=np.int64)
+    vocab_pos = np.asarray(vocab_pos, dtype=np.int64)
+    V = vocab_pos.size
+    if prefix_table.size != V:
+        raise OracleError("invalid_arg", f"prefix table of {prefix_table.size} entries, V={V}")
+    if ((targets < -1) | (targets >= V)).any():
+        raise OracleError("bad_index", "target outside [-1, V)")
+    if ((prefix_table < -1) | (prefix_table >= V)).any():
+        raise OracleError("bad_index", "prefix class outside [-1, V)")
+    pos = np.append(vocab_pos, -1)  # entry V: the "no prefix" sentinel
+    valid = targets >= 0
+    prefix_targets = np.full(targets.shape, -1, dtype=np.int64)
+    prefix_targets[valid] = prefix_table[targets[valid]]
+    return pos[prefix_targets]  # -1 indexes the sentinel
+
+
 # ---------------------------------------------------------------------------
 # Loss and gradients (floating-point part)
 # ---------------------------------------------------------------------------

@@ -32,7 +32,8 @@ EXPORTS = (
     "ss_workspace_bytes", "ss_build_workspace_bytes", "ss_build_candidates",
     "ss_build_candidates_noalloc", "ss_ce_forward", "ss_ce_backward",
     "ss_status_string", "ss_last_cuda_error", "ss_version", "ss_timing_enable",
-    "ss_timing_reset", "ss_timing_count", "ss_timing_query",
+    "ss_timing_reset", "ss_timing_count", "ss_timing_query", "ss_prefix_positions",
+    "ss_selftest_wait_limit",
 )
 
 
@@ -74,6 +75,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ss_ce_forward": (_i32, [_p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _p, _sz, _p]),
         "ss_ce_backward": (_i32, [_p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _sz,
                                   _p]),
+        "ss_prefix_positions": (_i32, [_p, _p, _p, _i64, _i32, _p, _p, _p]),
+        "ss_selftest_wait_limit": (_i32, [_p, _p]),
         "ss_status_string": (ctypes.c_char_p, [_i32]),
         "ss_last_cuda_error": (ctypes.c_char_p, []),
         "ss_version": (_i32, []),
@@ -157,6 +160,20 @@ def ss_ce_backward(grad_loss, candidates, vocab_pos, n_valid, T, d, V, P, dx, dW
         _ptr(grad_loss), _ptr(candidates), _ptr(vocab_pos), _ptr(n_valid), T, d, V, P, _ptr(dx), _ptr(dW), _ptr(dev_status), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check("ss_ce_backward", code)
+
+
+def ss_prefix_positions(prefix_table, targets, vocab_pos, V, prefix_pos, dev_status, stream=None):
+    """prefix_pos[i] = position in C of prefix_table[targets[i]], -1 if absent."""
+    code = load().ss_prefix_positions(
+        _ptr(prefix_table), _ptr(targets), _ptr(vocab_pos), targets.numel(), V, _ptr(prefix_pos),
+        _ptr(dev_status), _stream(stream))
+    _check("ss_prefix_positions", code)
+
+
+def ss_selftest_wait_limit(dev_status, stream=None):
+    """Run one kernel wait out on purpose; the outcome lands in dev_status[8..11]."""
+    _check("ss_selftest_wait_limit", load().ss_selftest_wait_limit(_ptr(dev_status),
+                                                                    _stream(stream)))
 
 
 def ss_status_string(code: int) -> str:

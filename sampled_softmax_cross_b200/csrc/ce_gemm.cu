@@ -17,8 +17,9 @@
 // ("Learning Triton One Kernel at a Time: Softmax": max-shifted softmax and
 // the tile-wise sum of its "Online Softmax" section, with the target logit as
 // the shift). Because loss_i = lse_i - z_target >= max_j z_ij - z_target, E
-// can only overflow on a row whose loss exceeds ~88 nats; such rows are
-// found from a non-finite S_i and recomputed exactly (ce_kernels.cu).
+// can only grow large on a row whose loss is large; rows whose S_i reaches
+// 2^64 (loss >= 44 nats) are recomputed exactly with the row maximum as the
+// shift (ce_kernels.cu).
 // After the forward, the row pass writes E'_{i,t_i} = 1 - S_i at the target
 // column, r_i = 1 / S_i and x'_i = r_i x_i, so that r_i E'_ij is exactly
 // softmax_ij - [j == t_i] (section "Gradient") and the backward is two plain
@@ -94,6 +95,44 @@ SS_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, 
   ok = __all_sync(0xffffffffu, ok);
   if (!ok) raise_abort(abort_flag, status, kind);
   return ok;
+}
+
+// Self-test of the bounded wait above, on one CTA of two warps. Warp 0 waits
+// on a barrier that nothing completes and, when the limit passes, raises the
+// abort flag and records SS_ERR_KERNEL_TIMEOUT -- what a GEMM warp does when
+// its pipeline stalls. Warp 1 begins its own wait on a second such barrier an
+// eighth of the limit later, so it must leave through the flag before its
+// own limit, as the other warps of a stalled GEMM do. status = dev_status + 8:
+// [0] error, [1] detail (100 + 7), [2] 1 if warp 1 left through the flag,
+// [3] warp 0's wait in milliseconds.
+__global__ void __launch_bounds__(64, 1) k_wait_selftest(int32_t* status) {
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_word;
+  volatile int* abort_flag = &abort_word;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    const unsigned long long t = globaltimer();
+    while (globaltimer() - t < kWaitLimitNs / 8) __nanosleep(1000);
+  }
+  const unsigned long long t0 = globaltimer();
+  const bool ok = warp_wait(&bars[warp], 0u, abort_flag, status, 7);
+  const unsigned long long waited = globaltimer() - t0;
+  if (lane == 0) {
+    if (warp == 0) status[3] = (int32_t)(waited / 1000000ull);
+    if (warp == 1) status[2] = (!ok && waited < kWaitLimitNs) ? 1 : 0;
+  }
+}
+
+cudaError_t launch_wait_selftest(int32_t* status, cudaStream_t s) {
+  k_wait_selftest<<<1, 64, 0, s>>>(status);
+  return cudaGetLastError();
 }
 
 template <int KIND>

@@ -570,6 +570,35 @@ __global__ void k_zero_rows(uint4* __restrict__ dW, int32_t V, int32_t vec_per_r
 }
 
 // ----------------------------------------------------------------------------
+// Prefix-target positions (sampled_softmax.py, CandidateBuilder.build: the
+// prefix target of each token, then its position in C through the same
+// class -> position map as the targets). One thread per token; a prefix class
+// outside C, "no prefix" (-1) and an ignored token all give -1, so a prefix
+// target never adds a class to C.
+// ----------------------------------------------------------------------------
+__global__ void k_prefix_pos(const int32_t* __restrict__ prefix_table,
+                             const int32_t* __restrict__ targets,
+                             const int32_t* __restrict__ vocab_pos, int64_t T, int32_t V,
+                             int32_t* __restrict__ prefix_pos, int32_t* __restrict__ status) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < T; i += stride) {
+    const int t = __ldg(targets + i);
+    int pos = -1, bad = 0;
+    if (t >= 0 && t < V) {
+      const int p = __ldg(prefix_table + t);
+      if (p >= 0 && p < V)
+        pos = __ldg(vocab_pos + p);
+      else if (p != -1)
+        bad = 2;
+    } else if (t != -1) {
+      bad = 3;
+    }
+    if (bad && atomicCAS(status, 0, (int32_t)SS_ERR_BAD_INDEX) == 0) status[1] = bad;
+    prefix_pos[i] = pos;
+  }
+}
+
+// ----------------------------------------------------------------------------
 // launchers
 // ----------------------------------------------------------------------------
 static int g_sms_cache = 0;
@@ -650,6 +679,15 @@ cudaError_t launch_fixup(const RowArgs& a, cudaStream_t s) {
 cudaError_t launch_finalize(const float* loss_rows, const int32_t* tpos, int64_t T, int32_t P,
                             float* loss, int32_t* n_valid, cudaStream_t s) {
   k_finalize<<<1, 1024, 0, s>>>(loss_rows, tpos, T, P, loss, n_valid);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefix_pos(const int32_t* prefix_table, const int32_t* targets,
+                              const int32_t* vocab_pos, int64_t T, int32_t V, int32_t* prefix_pos,
+                              int32_t* status, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = (int)min64((T + 255) / 256, (int64_t)num_sms() * 8);
+  k_prefix_pos<<<blocks, 256, 0, s>>>(prefix_table, targets, vocab_pos, T, V, prefix_pos, status);
   return cudaGetLastError();
 }
 

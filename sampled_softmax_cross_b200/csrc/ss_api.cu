@@ -415,6 +415,32 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   return SS_OK;
 }
 
+ss_status ss_prefix_positions(const int32_t* prefix_table, const int32_t* targets,
+                              const int32_t* vocab_pos, int64_t T, int32_t V, int32_t* prefix_pos,
+                              int32_t* dev_status, void* stream) {
+  if (T < 0 || T > INT32_MAX || V < 1 || V > SS_MAX_VOCAB) return SS_ERR_INVALID_ARG;
+  if (prefix_table == nullptr || vocab_pos == nullptr || dev_status == nullptr ||
+      (T > 0 && (targets == nullptr || prefix_pos == nullptr)))
+    return SS_ERR_INVALID_ARG;
+  int sms;
+  ss_status ds = ensure_device(&sms);
+  if (ds != SS_OK) return ds;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  SS_LAUNCH("prefix_pos", s,
+            launch_prefix_pos(prefix_table, targets, vocab_pos, T, V, prefix_pos, dev_status + 8, s));
+  return SS_OK;
+}
+
+ss_status ss_selftest_wait_limit(int32_t* dev_status, void* stream) {
+  if (dev_status == nullptr) return SS_ERR_INVALID_ARG;
+  int sms;
+  ss_status ds = ensure_device(&sms);
+  if (ds != SS_OK) return ds;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  SS_LAUNCH("wait_selftest", s, launch_wait_selftest(dev_status + 8, s));
+  return SS_OK;
+}
+
 ss_status ss_timing_enable(int32_t enable) {
   g_tm.on = enable != 0;
   return SS_OK;

@@ -41,6 +41,8 @@ cudaError_t launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b,
 int gemm_smem_bytes(int kind);
 const void* gemm_kernel_ptr(int kind);
 int gemm_max_pairs(int kind, int sms);
+// One CTA that runs the pipelines' bounded wait out on purpose (ce_gemm.cu).
+cudaError_t launch_wait_selftest(int32_t* status, cudaStream_t s);
 
 // Small kernels (ce_kernels.cu). Each returns the launch error.
 cudaError_t launch_build_mark(const int32_t* targets, int64_t T, int32_t V, int32_t P,
@@ -78,6 +80,10 @@ cudaError_t launch_rows(const RowArgs& a, cudaStream_t s);
 cudaError_t launch_fixup(const RowArgs& a, cudaStream_t s);
 cudaError_t launch_finalize(const float* loss_rows, const int32_t* tpos, int64_t T, int32_t P,
                             float* loss, int32_t* n_valid, cudaStream_t s);
+// prefix_pos[i] = position in C of prefix_table[targets[i]], -1 if none.
+cudaError_t launch_prefix_pos(const int32_t* prefix_table, const int32_t* targets,
+                              const int32_t* vocab_pos, int64_t T, int32_t V, int32_t* prefix_pos,
+                              int32_t* status, cudaStream_t s);
 cudaError_t launch_zero_rows(uint16_t* dW, int32_t V, int32_t d, const int32_t* vocab_pos,
                              int all_rows, cudaStream_t s);
 

@@ -121,3 +121,15 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(capi, "_lib", None)
     with pytest.raises(capi.LibraryNotBuilt):
         capi.load(str(tmp_path / "nope.so"))
+
+
+def test_prefix_and_selftest_host_rejections(lib):
+    a = ctypes.c_void_p(1 << 20)  # never dereferenced: rejected before any CUDA call
+    f = lib.ss_prefix_positions
+    assert f(a, a, a, 10, 0, a, a, None) == capi.STATUS["SS_ERR_INVALID_ARG"]  # V < 1
+    assert f(a, a, a, -1, 100, a, a, None) == capi.STATUS["SS_ERR_INVALID_ARG"]  # T < 0
+    assert f(a, a, a, 10, capi.MAX_VOCAB + 1, a, a, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    assert f(None, a, a, 10, 100, a, a, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    assert f(a, None, a, 10, 100, a, a, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    assert f(a, a, a, 10, 100, a, None, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    assert lib.ss_selftest_wait_limit(None, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
