@@ -64,6 +64,26 @@ def peaks():
 
 # ---------------------------------------------------------------- clocks --
 
+# Dense bf16 tensor-core work per SM per clock on sm_100 (4096 FMA): 148 SMs at
+# the 1.86 GHz boost give the 2.25 PFLOP/s datasheet figure.
+BF16_FLOP_PER_CLK_SM = 8192
+NUM_SMS = 148
+
+
+def clock_normalized(step_tflops, per, clk, world):
+    """The step's and the GEMMs' TFLOP/s against the tensor peak at the SM clock
+    seen during the timed region (the 1 kW power cap moves that clock from box
+    to box; this ratio does not move with it)."""
+    if not clk or not clk.get("sm_mhz"):
+        return None
+    peak = BF16_FLOP_PER_CLK_SM * NUM_SMS * clk["sm_mhz"] * 1e6 / 1e12 * world
+    out = {"sm_mhz": clk["sm_mhz"], "tensor_peak_tflops_at_clock": peak,
+           "step_frac": step_tflops / peak}
+    for k in ("fwd_gemm_ce", "dx_gemm", "dw_gemm_scatter"):
+        if k in per and "tflops" in per[k]:
+            out[k + "_frac"] = per[k]["tflops"] / (peak / world)
+    return out
+
 class ClockSampler:
     """nvidia-smi clock and throttle-reason samples taken while the timed region runs."""
 
@@ -383,6 +403,9 @@ def run_ours(args, w):
             "dw_gemm_scatter": ("tensor", flops_gemm),
             "gather": ("hbm", 2.0 * w.P * w.d * 2),
             "zero_rows": ("hbm", (w.V - w.P) * w.d * 2.0 + w.V * 4),
+            "ref_logits": ("hbm", 2.0 * w.T * w.d * 2 + w.T * 4.0 * 2),
+            "row_pass": ("hbm", ((w.P + 255) // 256) * w.T * 4.0 + 2.0 * w.T * w.d * 2
+                         + w.T * 4.0 * 5),
             "build_mark": ("hbm", w.T * 4.0 + 2 * ((w.V + 31) // 32) * 4),
             "build_emit": ("hbm", w.T * 4.0 * 2 + w.V * 4.0 * 2 + w.P * 4.0),
         }
@@ -449,6 +472,7 @@ def run_ours(args, w):
             "kernels": per,
             "gpu_launches": launches,
             "clocks": clk,
+            "clock_normalized": clock_normalized(step_tflops, per, clk, world),
             "e2e": e2e,
             "cpu_baseline": cpu,
         }

@@ -289,6 +289,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       const int nv = __ldg(args.n_valid);
       scale = nv > 0 ? __ldg(args.grad_loss) / (float)nv : 0.f;
     }
+    if (KIND == KIND_DW && args.vocab_pos != nullptr) {
+      // The rows of dW outside C are +0.0. The epilogue warps of every CTA
+      // write them while the first tiles' MMAs run (they are disjoint from
+      // the rows the tiles scatter). Each warp takes blocks of 32 classes.
+      const int vpr = args.N / 8;
+      const int64_t gw = (int64_t)blockIdx.x * 4 + e, nw = (int64_t)gridDim.x * 4;
+      uint4* dW4 = reinterpret_cast<uint4*>(args.dW);
+      for (int64_t base = gw * 32; base < args.V; base += nw * 32) {
+        const int64_t r = base + lane;
+        const bool zero_row = r < args.V && __ldg(args.vocab_pos + r) < 0;
+        unsigned m = __ballot_sync(0xffffffffu, zero_row);
+        while (m) {
+          const int k = __ffs(m) - 1;
+          m &= m - 1;
+          uint4* dst = dW4 + (base + k) * vpr;
+          for (int v = lane; v < vpr; v += 32) __stcs(dst + v, make_uint4(0, 0, 0, 0));
+        }
+      }
+    }
     for (int tile = cluster; tile < num_tiles; tile += num_clusters, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;

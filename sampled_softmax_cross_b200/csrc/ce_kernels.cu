@@ -375,11 +375,14 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 a, float r) {
 // all their loads in flight.
 constexpr int kRowsPerWarp = 8;
 
-__global__ void k_rows(RowArgs a) {
+__global__ void __launch_bounds__(256) k_rows(RowArgs a) {
+  __shared__ double2 s_part[8];
   const int lane = threadIdx.x & 31;
   const int vpr = a.d / 8;
   const int64_t groups = (a.T + kRowsPerWarp - 1) / kRowsPerWarp;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  double w_sum = 0.0;  // this warp's valid, non-overflowed row losses (lane 0)
+  int w_cnt = 0;       // this warp's valid rows
   for (int64_t gidx = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); gidx < groups;
        gidx += warps) {
     const int64_t r = gidx * kRowsPerWarp + (lane & 7);
@@ -402,6 +405,17 @@ __global__ void k_rows(RowArgs a) {
         a.rscale[r] = rs;
         if (valid) a.u[r * a.ldz + tp] = (uint16_t)(pack_bf16x2(1.f - S, 0.f) & 0xffffu);
       }
+    }
+    {  // loss sum and valid count of the warp's 8 rows, fixed order
+      double l = (lane < 8 && in && valid && !fix) ? (double)logf(S) : 0.0;
+      int c = (lane < 8 && in && valid) ? 1 : 0;
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        l += __shfl_xor_sync(0xffffffffu, l, o);
+        c += __shfl_xor_sync(0xffffffffu, c, o);
+      }
+      w_sum += l;
+      w_cnt += c;
     }
     const unsigned todo = __ballot_sync(0xffffffffu, lane < 8 && in && !fix);
     for (int k0 = 0; k0 < kRowsPerWarp; k0 += 4) {
@@ -432,12 +446,27 @@ __global__ void k_rows(RowArgs a) {
       }
     }
   }
+  if (lane == 0) s_part[threadIdx.x >> 5] = make_double2(w_sum, (double)w_cnt);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double2 t = s_part[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+      t.x += s_part[w].x;
+      t.y += s_part[w].y;
+    }
+    a.partials[blockIdx.x] = t;
+  }
 }
 
-// Exact recomputation of listed rows, max-shifted (section "Definition"):
-// one CTA per row recomputes the row's P logits in fp32, then rewrites lse,
-// the row loss, r_i, x'_i and the row of E' with the row max as the shift.
-constexpr int kFixThreads = 256;
+// After the row pass, one CTA:
+//  1. exact recomputation of listed rows, max-shifted (section "Definition"):
+//     the row's P logits in fp32, then lse, the row loss, r_i, x'_i and the
+//     row of E' with the row max as the shift;
+//  2. the loss: sum of the valid rows' losses over the valid-row count
+//     (Handout #16 CPU checks, lm_gradient), in a fixed order (deterministic).
+//     Without listed rows it adds the row pass's per-block partial sums; with
+//     them it adds every row's loss again.
+constexpr int kFinThreads = 1024;
 
 __device__ float block_reduce(float v, bool is_max, float* sh) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -450,7 +479,7 @@ __device__ float block_reduce(float v, bool is_max, float* sh) {
   __syncthreads();
   if (threadIdx.x == 0) {
     float t = sh[0];
-    for (int w = 1; w < kFixThreads / 32; ++w) t = is_max ? fmaxf(t, sh[w]) : t + sh[w];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) t = is_max ? fmaxf(t, sh[w]) : t + sh[w];
     sh[32] = t;
   }
   __syncthreads();
@@ -465,24 +494,25 @@ __device__ __forceinline__ float row_logit(const uint4* xr, const uint4* wr, int
   return acc;
 }
 
-__global__ void __launch_bounds__(kFixThreads) k_fixup(RowArgs a) {
+__global__ void __launch_bounds__(kFinThreads) k_finalize(RowArgs a, int32_t nparts) {
   __shared__ float sh[33];
   __shared__ float s_zt;
+  __shared__ double s_sum[32], s_cnt[32];
   const int n = *reinterpret_cast<volatile int32_t*>(a.fix_count);
   const int vpr = a.d / 8;
-  for (int k = blockIdx.x; k < n; k += gridDim.x) {
+  const int nt = blockDim.x;
+  for (int k = 0; k < n; ++k) {
     const int64_t r = a.fix_list[k];
     const int tp = a.tpos[r];
     const bool valid = tp >= 0 && tp < a.P;
     const uint4* xr = reinterpret_cast<const uint4*>(a.x) + r * vpr;
     const uint4* w = reinterpret_cast<const uint4*>(a.w_c);
     float m = -INFINITY;
-    for (int j = threadIdx.x; j < a.P; j += kFixThreads)
-      m = fmaxf(m, row_logit(xr, w + (int64_t)j * vpr, vpr));
+    for (int j = threadIdx.x; j < a.P; j += nt) m = fmaxf(m, row_logit(xr, w + (int64_t)j * vpr, vpr));
     m = block_reduce(m, true, sh);
     float sum = 0.f;
     uint16_t* ur = a.u + r * a.ldz;
-    for (int j = threadIdx.x; j < a.P; j += kFixThreads) {
+    for (int j = threadIdx.x; j < a.P; j += nt) {
       const float z = row_logit(xr, w + (int64_t)j * vpr, vpr);
       const float e = expf(z - m);
       sum += e;
@@ -499,41 +529,41 @@ __global__ void __launch_bounds__(kFixThreads) k_fixup(RowArgs a) {
       if (valid) ur[tp] = (uint16_t)(pack_bf16x2(expf(s_zt - m) - S, 0.f) & 0xffffu);
     }
     uint4* xo = reinterpret_cast<uint4*>(a.xs) + r * vpr;
-    for (int v = threadIdx.x; v < vpr; v += kFixThreads) xo[v] = scale_bf16x8(__ldg(xr + v), rs);
+    for (int v = threadIdx.x; v < vpr; v += nt) xo[v] = scale_bf16x8(__ldg(xr + v), rs);
     __syncthreads();
   }
-}
 
-// ----------------------------------------------------------------------------
-// Loss: sum of the valid rows' losses over the valid-row count (Handout #16
-// CPU checks, lm_gradient), in a fixed order (deterministic).
-// ----------------------------------------------------------------------------
-__global__ void k_finalize(const float* __restrict__ loss_rows, const int32_t* __restrict__ tpos,
-                           int64_t T, int32_t P, float* __restrict__ loss,
-                           int32_t* __restrict__ n_valid) {
-  __shared__ double s_sum[32], s_cnt[32];
   double s = 0.0, c = 0.0;
-  // each thread takes runs of 4 consecutive rows (T rounded down to a multiple
-  // of 4 here; the rest below), fixed order
-  const int64_t T4 = T & ~int64_t(3);
-  for (int64_t i = 4 * (int64_t)threadIdx.x; i < T4; i += 4 * (int64_t)blockDim.x) {
-    const float4 l = __ldg(reinterpret_cast<const float4*>(loss_rows + i));
-    const int4 t = __ldg(reinterpret_cast<const int4*>(tpos + i));
-    const float lv[4] = {l.x, l.y, l.z, l.w};
-    const int tv[4] = {t.x, t.y, t.z, t.w};
+  if (n == 0) {
+    for (int i = threadIdx.x; i < nparts; i += nt) {
+      const double2 p = a.partials[i];
+      s += p.x;
+      c += p.y;
+    }
+  } else {
+    // each thread takes runs of 4 consecutive rows (T rounded down to a
+    // multiple of 4 here; the rest below), fixed order
+    const int64_t T = a.T;
+    const int64_t T4 = T & ~int64_t(3);
+    for (int64_t i = 4 * (int64_t)threadIdx.x; i < T4; i += 4 * (int64_t)nt) {
+      const float4 l = *reinterpret_cast<const float4*>(a.loss_rows + i);
+      const int4 t = __ldg(reinterpret_cast<const int4*>(a.tpos + i));
+      const float lv[4] = {l.x, l.y, l.z, l.w};
+      const int tv[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (tv[u] >= 0 && tv[u] < P) {
-        s += (double)lv[u];
-        c += 1.0;
+      for (int u = 0; u < 4; ++u) {
+        if (tv[u] >= 0 && tv[u] < a.P) {
+          s += (double)lv[u];
+          c += 1.0;
+        }
       }
     }
-  }
-  for (int64_t i = T4 + threadIdx.x; i < T; i += blockDim.x) {
-    const int t = tpos[i];
-    if (t >= 0 && t < P) {
-      s += (double)loss_rows[i];
-      c += 1.0;
+    for (int64_t i = T4 + threadIdx.x; i < T; i += nt) {
+      const int t = a.tpos[i];
+      if (t >= 0 && t < a.P) {
+        s += (double)a.loss_rows[i];
+        c += 1.0;
+      }
     }
   }
 #pragma unroll
@@ -548,12 +578,12 @@ __global__ void k_finalize(const float* __restrict__ loss_rows, const int32_t* _
   __syncthreads();
   if (threadIdx.x == 0) {
     double ts = 0.0, tc = 0.0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+    for (int w = 0; w < (nt >> 5); ++w) {
       ts += s_sum[w];
       tc += s_cnt[w];
     }
-    *n_valid = (int32_t)tc;
-    *loss = tc > 0.0 ? (float)(ts / tc) : 0.f;
+    *a.n_valid = (int32_t)tc;
+    *a.loss = tc > 0.0 ? (float)(ts / tc) : 0.f;
   }
 }
 
@@ -660,25 +690,21 @@ cudaError_t launch_ref_logits(const uint16_t* x, const uint16_t* w_c, const int3
   return cudaGetLastError();
 }
 
+static int rows_blocks(int64_t T) {
+  if (T == 0) return 0;
+  const int64_t groups = (T + kRowsPerWarp - 1) / kRowsPerWarp;  // per warp; 8 warps per block
+  return (int)min64(min64((groups + 7) / 8, (int64_t)num_sms() * 16), (int64_t)kRowPartials);
+}
+
 cudaError_t launch_rows(const RowArgs& a, cudaStream_t s) {
-  if (a.T == 0) return cudaSuccess;
-  const int64_t groups = (a.T + kRowsPerWarp - 1) / kRowsPerWarp;  // per warp; 8 warps per block
-  const int blocks = (int)min64((groups + 7) / 8, (int64_t)num_sms() * 16);
+  const int blocks = rows_blocks(a.T);
+  if (blocks == 0) return cudaSuccess;
   k_rows<<<blocks, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_fixup(const RowArgs& a, cudaStream_t s) {
-  if (a.T == 0) return cudaSuccess;
-  // Rows are flagged only when their loss is enormous, so one CTA (which
-  // finds the list empty in the common case) is enough.
-  k_fixup<<<1, kFixThreads, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_finalize(const float* loss_rows, const int32_t* tpos, int64_t T, int32_t P,
-                            float* loss, int32_t* n_valid, cudaStream_t s) {
-  k_finalize<<<1, 1024, 0, s>>>(loss_rows, tpos, T, P, loss, n_valid);
+cudaError_t launch_finalize(const RowArgs& a, cudaStream_t s) {
+  k_finalize<<<1, kFinThreads, 0, s>>>(a, rows_blocks(a.T));
   return cudaGetLastError();
 }
 

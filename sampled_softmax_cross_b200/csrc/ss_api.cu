@@ -153,7 +153,8 @@ constexpr int kBM = 128, kBN = 256, kBMP = 256;  // rows per CTA, cols per tile,
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-  size_t bitmap, prefix, ref, rscale, loss_rows, fix_list, fix_count, w_c, u, rowsum, xs, total;
+  size_t bitmap, prefix, ref, rscale, loss_rows, fix_list, fix_count, partials, w_c, u, rowsum, xs,
+      total;
   int64_t ldz;
   int tiles_n;
 };
@@ -182,6 +183,7 @@ Layout layout(int64_t T, int32_t d, int32_t V, int32_t P) {
   L.loss_rows = take((size_t)T * 4, 256);
   L.fix_list = take((size_t)T * 4, 256);
   L.fix_count = take(16, 256);
+  L.partials = take((size_t)kRowPartials * sizeof(double2), 256);
   L.w_c = take((size_t)P * d * 2, 1024);
   L.u = take((size_t)T * L.ldz * 2, 1024);
   L.rowsum = take((size_t)L.tiles_n * T * 4, 1024);
@@ -293,6 +295,28 @@ ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t*
   int32_t* fix_count = reinterpret_cast<int32_t*>(ws + L.fix_count);
   int32_t* kstatus = dev_status + 8;
 
+  RowArgs ra{};
+  ra.rowsum = rowsum;
+  ra.ref = ref;
+  ra.tpos = target_pos;
+  ra.x = x;
+  ra.T = T;
+  ra.d = d;
+  ra.P = P;
+  ra.tiles_n = L.tiles_n;
+  ra.ldz = L.ldz;
+  ra.w_c = w_c;
+  ra.u = u;
+  ra.lse = lse;
+  ra.rscale = reinterpret_cast<float*>(ws + L.rscale);
+  ra.xs = reinterpret_cast<uint16_t*>(ws + L.xs);
+  ra.loss_rows = loss_rows;
+  ra.fix_list = reinterpret_cast<int32_t*>(ws + L.fix_list);
+  ra.fix_count = fix_count;
+  ra.partials = reinterpret_cast<double2*>(ws + L.partials);
+  ra.loss = loss;
+  ra.n_valid = n_valid;
+
   SS_LAUNCH("gather", s, launch_gather(lm_head, candidates, P, d, V, w_c, kstatus, fix_count, 1, s));
   if (T > 0) {
     SS_LAUNCH("ref_logits", s, launch_ref_logits(x, w_c, target_pos, T, d, P, ref, s));
@@ -317,28 +341,9 @@ ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t*
     const int tiles = a.tiles_m * a.tiles_n;
     SS_LAUNCH("fwd_gemm_ce", s,
               launch_gemm(KIND_FWD, ta, tb, tc, a, tiles < pairs[KIND_FWD] ? tiles : pairs[KIND_FWD], s));
-    RowArgs ra{};
-    ra.rowsum = rowsum;
-    ra.ref = ref;
-    ra.tpos = target_pos;
-    ra.x = x;
-    ra.T = T;
-    ra.d = d;
-    ra.P = P;
-    ra.tiles_n = L.tiles_n;
-    ra.ldz = L.ldz;
-    ra.w_c = w_c;
-    ra.u = u;
-    ra.lse = lse;
-    ra.rscale = reinterpret_cast<float*>(ws + L.rscale);
-    ra.xs = reinterpret_cast<uint16_t*>(ws + L.xs);
-    ra.loss_rows = loss_rows;
-    ra.fix_list = reinterpret_cast<int32_t*>(ws + L.fix_list);
-    ra.fix_count = fix_count;
     SS_LAUNCH("row_pass", s, launch_rows(ra, s));
-    SS_LAUNCH("row_fixup", s, launch_fixup(ra, s));
   }
-  SS_LAUNCH("loss_finalize", s, launch_finalize(loss_rows, target_pos, T, P, loss, n_valid, s));
+  SS_LAUNCH("loss_finalize", s, launch_finalize(ra, s));
   return SS_OK;
 }
 
@@ -369,7 +374,6 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
     SS_LAUNCH("zero_rows", s, launch_zero_rows(dW, V, d, vocab_pos, 1, s));
     return SS_OK;
   }
-  SS_LAUNCH("zero_rows", s, launch_zero_rows(dW, V, d, vocab_pos, 0, s));
 
   CUtensorMap ua, wb, dxs, ua2, xb;
   ss_status r;
@@ -392,7 +396,7 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   a.out = dx;
   a.ld_out = d;
   a.status = kstatus;
-  int tiles = a.tiles_m * a.tiles_n;
+  const int tiles = a.tiles_m * a.tiles_n;
   SS_LAUNCH("dx_gemm", s,
             launch_gemm(KIND_DX, ua, wb, dxs, a, tiles < pairs[KIND_DX] ? tiles : pairs[KIND_DX], s));
 
@@ -406,12 +410,12 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   b.cand = candidates;
   b.dW = dW;
   b.V = V;
+  b.vocab_pos = vocab_pos;  // the epilogue warps also zero the rows outside C
   b.grad_loss = grad_loss;
   b.n_valid = n_valid;
   b.status = kstatus;
-  tiles = b.tiles_m * b.tiles_n;
-  SS_LAUNCH("dw_gemm_scatter", s,
-            launch_gemm(KIND_DW, ua2, xb, ua2, b, tiles < pairs[KIND_DW] ? tiles : pairs[KIND_DW], s));
+  // every resident pair, even without a tile, so that the zero rows are spread over all SMs
+  SS_LAUNCH("dw_gemm_scatter", s, launch_gemm(KIND_DW, ua2, xb, ua2, b, pairs[KIND_DW], s));
   return SS_OK;
 }
 

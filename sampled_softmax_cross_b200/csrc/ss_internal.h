@@ -27,9 +27,10 @@ struct GemmArgs {
   uint16_t* out;        // [M][ld_out] bf16 (E for the forward, dx for dX)
   int64_t ld_out;
   // dW epilogue
-  const int32_t* cand;  // [M] class id of each output row
-  uint16_t* dW;         // [V][N] bf16
+  const int32_t* cand;       // [M] class id of each output row
+  uint16_t* dW;              // [V][N] bf16
   int32_t V;
+  const int32_t* vocab_pos;  // [V] (dW) rows with -1 are set to +0.0 by the epilogue warps
   int32_t* status;  // dev_status + 8 (error word, detail word)
 };
 
@@ -75,11 +76,15 @@ struct RowArgs {
   float* loss_rows;     // [T]
   int32_t* fix_list;    // [T] rows whose E overflowed
   int32_t* fix_count;   // [1]
+  double2* partials;    // [kRowPartials] per-block (loss sum, valid count) of the row pass
+  float* loss;          // [1] mean loss over valid rows
+  int32_t* n_valid;     // [1]
 };
+// Most blocks the row pass launches (the size of RowArgs::partials).
+constexpr int kRowPartials = 4096;
 cudaError_t launch_rows(const RowArgs& a, cudaStream_t s);
-cudaError_t launch_fixup(const RowArgs& a, cudaStream_t s);
-cudaError_t launch_finalize(const float* loss_rows, const int32_t* tpos, int64_t T, int32_t P,
-                            float* loss, int32_t* n_valid, cudaStream_t s);
+// Exact recomputation of overflowed rows, then the loss mean (one CTA).
+cudaError_t launch_finalize(const RowArgs& a, cudaStream_t s);
 // prefix_pos[i] = position in C of prefix_table[targets[i]], -1 if none.
 cudaError_t launch_prefix_pos(const int32_t* prefix_table, const int32_t* targets,
                               const int32_t* vocab_pos, int64_t T, int32_t V, int32_t* prefix_pos,

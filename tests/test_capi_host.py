@@ -63,8 +63,10 @@ def test_workspace_bytes_rejects_bad_sizes(lib):
 def test_workspace_holds_logits_and_rows(lib):
     T, d, V, P = 49152, 768, 50304, 24576
     ws = capi.ss_workspace_bytes(T, d, V, P)
-    # E' [T,P] + W_C [P,d] + x' [T,d] (bf16), tile sums, per-row words, builder bitmap
-    need = T * P * 2 + P * d * 2 + T * d * 2 + ((P + 255) // 256) * T * 4 + 4 * T * 4
+    # E' [T,P] + W_C [P,d] + x' [T,d] (bf16), tile sums, per-row words, the row
+    # pass's per-block partial sums (4096 x 16 B), builder bitmap
+    need = (T * P * 2 + P * d * 2 + T * d * 2 + ((P + 255) // 256) * T * 4 + 4 * T * 4
+            + 4096 * 16)
     assert need <= ws <= need + 2 * ((V + 31) // 32) * 4 + 64 * 1024
     # padded logit rows when P is not a multiple of 8
     assert capi.ss_workspace_bytes(100, 64, 5000, 1001) >= 100 * 1008 * 2
