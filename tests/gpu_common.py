@@ -5,7 +5,10 @@ oracle on the same seeded inputs, and holds the tolerances:
 
 * candidate set, target/vocab positions, builder info, dW zero pattern:
   bit-exact;
-* loss: relative 1e-3; lse: absolute 1e-3 (both come from fp32 accumulators);
+* loss: relative 1e-3, plus an absolute 1e-6 for losses at or near 0 (P = 1,
+  where the exact loss is 0 and the GPU's is the log of 1 + the fp32 rounding
+  difference between the tensor-core logit and the fp32 target logit);
+  lse: absolute 1e-3 (both come from fp32 accumulators);
 * dX and dW (rows in C): relative Frobenius error 2e-2 (bf16 outputs from bf16
   logits), with max-abs error / max |expected| reported.
 """
@@ -20,6 +23,7 @@ from sampled_softmax_cross_b200 import capi
 from sampled_softmax_cross_b200 import workloads as wl
 
 LOSS_RTOL = 1e-3
+LOSS_ATOL = 1e-6
 LSE_ATOL = 1e-3
 GRAD_RTOL = 2e-2
 
@@ -90,7 +94,8 @@ def compare_full(g: dict, o: dict, targets: np.ndarray):
     assert np.array_equal(g["vocab_pos"], o["vocab_pos"])
     assert g["n_valid"] == o["n_valid"]
     if o["n_valid"]:
-        assert abs(g["loss"] - o["loss"]) <= LOSS_RTOL * abs(o["loss"]), (g["loss"], o["loss"])
+        assert abs(g["loss"] - o["loss"]) <= LOSS_RTOL * abs(o["loss"]) + LOSS_ATOL, (g["loss"],
+                                                                                   o["loss"])
     else:
         assert g["loss"] == 0.0
     if targets.size:

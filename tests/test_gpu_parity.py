@@ -135,6 +135,44 @@ def test_small_shapes_match_oracle(T, d, V, P, seed, grad):
     compare_full(g, o, t)
 
 
+def _edge_case(kind):
+    rng = np.random.default_rng(hash(kind) % (1 << 32))
+    if kind == "one_token":
+        x, lm, t = random_case(1, 64, 1000, 10, 21)
+        return x, lm, t, 10, 3
+    if kind == "one_class":  # P = 1: C = {the only target}; softmax 1, loss 0, gradients 0
+        x, lm, _ = wl.make_inputs(200, 64, 500, 1.1, 0.0, 22)
+        t = np.full(200, 7, np.int32)
+        t[::9] = -1
+        return x, lm, t, 1, 11
+    if kind == "one_target_class":  # D = 1, P - 1 negatives
+        x, lm, _ = wl.make_inputs(300, 96, 2000, 1.1, 0.0, 23)
+        return x, lm, np.full(300, 1234, np.int32), 300, 5
+    if kind == "wide_d":  # K = 4096 in the forward: 64 K blocks per tile
+        x, lm, t = random_case(256, 4096, 3001, 700, 24)
+        return x, lm, t, 700, 17
+    if kind == "max_vocab":  # V = SS_MAX_VOCAB, P = V / 4
+        V = capi.MAX_VOCAB
+        x, lm, t = random_case(256, 64, V, V // 4, 25)
+        return x, lm, t, V // 4, 123457
+    if kind == "huge_offset":  # a 64-bit offset, reduced mod V
+        x, lm, t = random_case(500, 64, 5003, 1500, 26)
+        return x, lm, t, 1500, (1 << 40) + 5
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("kind", ["one_token", "one_class", "one_target_class", "wide_d",
+                                  "max_vocab", "huge_offset"])
+def test_edge_shapes_match_oracle(kind):
+    x, lm, t, P, off = _edge_case(kind)
+    g = run_path(x, lm, t, P, off)
+    o = oracle_run(x, lm, t, P, off)
+    compare_full(g, o, t)
+    if kind == "one_class":  # exactly 0 up to fp32 rounding of z_target - ref
+        assert abs(g["loss"]) <= 1e-6
+        assert np.max(np.abs(wl.bits_to_f64(g["dx_bits"]))) <= 1e-6
+
+
 def test_tiny_workload_matches_oracle():
     w = wl.WORKLOADS["tiny"]
     x, lm, t = wl.workload_inputs(w)
