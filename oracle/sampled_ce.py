@@ -249,17 +249,22 @@ def dlogits(z: np.ndarray, lse: np.ndarray, target_pos: np.ndarray, scale: float
 
 def sampled_ce_backward(grad_loss: float, x: np.ndarray, w_c: np.ndarray,
                         candidates: np.ndarray, target_pos: np.ndarray,
-                        lse: np.ndarray, V: int, chunk: int = 1024):
+                        lse: np.ndarray, V: int, chunk: int = 1024,
+                        logit_x: np.ndarray | None = None, logit_w: np.ndarray | None = None):
     """dX = G @ W_C and the dense lm_head gradient dW (zeros outside C).
 
     Module docstring of sampled_softmax.py: "two gradient GEMMs" and "the
     gradient for lm_head is dense over the vocabulary with zeros outside C".
     dW_C = G^T @ x is accumulated over row chunks; dW[C_j] = dW_C[j].
+    G comes from the logits z = logit_x @ logit_w^T, by default x and W_C
+    themselves (the e4m3 variant passes its quantized operands here).
 
     Returns (dx float64 [T,d], dW float64 [V,d]).
     """
     x = np.asarray(x, dtype=np.float64)
     w_c = np.asarray(w_c, dtype=np.float64)
+    lx = x if logit_x is None else np.asarray(logit_x, dtype=np.float64)
+    lw = w_c if logit_w is None else np.asarray(logit_w, dtype=np.float64)
     tpos = np.asarray(target_pos, dtype=np.int64)
     T, d = x.shape
     n = int((tpos >= 0).sum())
@@ -267,7 +272,7 @@ def sampled_ce_backward(grad_loss: float, x: np.ndarray, w_c: np.ndarray,
     dx = np.zeros((T, d))
     dw_c = np.zeros_like(w_c)
     for r0, r1 in _row_chunks(T, chunk):
-        z = x[r0:r1] @ w_c.T
+        z = lx[r0:r1] @ lw.T
         g = dlogits(z, lse[r0:r1], tpos[r0:r1], scale)
         dx[r0:r1] = g @ w_c
         dw_c += g.T @ x[r0:r1]
@@ -287,6 +292,111 @@ def sampled_ce(x, lm_head, targets, P, offset=0, stride=NEGATIVE_STRIDE, grad_lo
     dx, dW = sampled_ce_backward(grad_loss, x, w_c, cand, tpos, lse, V, chunk)
     return dict(candidates=cand, target_pos=tpos, vocab_pos=vpos, info=info, loss=loss,
                 lse=lse, loss_rows=loss_rows, n_valid=n, dx=dx, dW=dW)
+
+
+# ---------------------------------------------------------------------------
+# e4m3 variant: the logits GEMM on 8-bit floating-point operands
+# ---------------------------------------------------------------------------
+#
+# sampled_softmax.py keeps the candidate rows as float8 e4m3 (SampledLoss.rows,
+# rows_t) and runs the logits through torch._scaled_mm; the scales are not on
+# the page. Readings for this variant:
+#   * format: OCP 8-bit floating point, E4M3 -- 1 sign bit, 4 exponent bits
+#     (bias 7), 3 mantissa bits, subnormals below 2^-6, no infinities, the
+#     codes S.1111.111 are NaN, largest finite magnitude 448;
+#   * rounding: to nearest, ties to even, finite results saturate at +-448;
+#   * scale: one power of two per tensor (x, and W_C of the step): the
+#     smallest 2^k with amax * 2^-k <= 448, so scaling is exact and the codes
+#     are round(v * 2^-k); 2^0 for an all-zero tensor;
+#   * only the logits GEMM uses them: z = (x_q 2^kx)(w_q 2^kw)^T; the softmax,
+#     loss and G follow from that z, and the gradient GEMMs use the bf16 x and
+#     W_C as in the bf16 path (the page does not give G's precision).
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(code: int) -> float:
+    """Value of an e4m3 code from its bit fields (NaN for S.1111.111)."""
+    code = int(code) & 0xFF
+    sign = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 0xF and m == 0x7:
+        return math.nan
+    if e == 0:
+        return sign * (m / 8.0) * 2.0 ** -6
+    return sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+def e4m3_round(v: np.ndarray) -> np.ndarray:
+    """Round to the e4m3 grid: nearest, ties to even, saturating at +-448.
+
+    In the binade [2^e, 2^(e+1)) the grid spacing is 2^(e-3); below 2^-6 it
+    is 2^-9 (subnormals). Division by the spacing is exact (a power of two)
+    and numpy's round is half-to-even.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(a)  # a = f * 2^ex with f in [0.5, 1): floor(log2 a) = ex - 1
+    e = np.maximum(ex - 1, -6)
+    q = np.ldexp(1.0, e - 3)
+    r = np.minimum(np.round(a / q) * q, E4M3_MAX)
+    return np.where(np.signbit(v), -r, r)
+
+
+def e4m3_encode(r: np.ndarray) -> np.ndarray:
+    """Codes of values already on the e4m3 grid (e4m3_round's output)."""
+    r = np.asarray(r, dtype=np.float64)
+    a = np.abs(r)
+    sub = a < 2.0 ** -6
+    _, ex = np.frexp(np.where(sub, 1.0, a))
+    e = ex - 1
+    mant_norm = np.round((np.where(sub, 1.0, a) / np.ldexp(1.0, e) - 1.0) * 8.0)
+    exp_field = np.where(sub, 0, e + 7)
+    mant = np.where(sub, np.round(a / 2.0 ** -9), mant_norm)
+    code = (exp_field.astype(np.int64) << 3) | mant.astype(np.int64)
+    code = np.where(np.signbit(r), code | 0x80, code)
+    return code.astype(np.uint8)
+
+
+def e4m3_scale_exponent(amax: float) -> int:
+    """The k of the per-tensor scale 2^k: smallest k with amax <= 448 * 2^k."""
+    amax = float(amax)
+    if not amax > 0.0:
+        return 0
+    _, ex = math.frexp(amax)
+    k = ex - 9
+    while amax > math.ldexp(E4M3_MAX, k):
+        k += 1
+    while amax <= math.ldexp(E4M3_MAX, k - 1):
+        k -= 1
+    return k
+
+
+def quantize_e4m3(a: np.ndarray):
+    """Per-tensor e4m3 quantization: (codes uint8, k, dequantized float64)."""
+    a = np.asarray(a, dtype=np.float64)
+    k = e4m3_scale_exponent(np.max(np.abs(a)) if a.size else 0.0)
+    r = e4m3_round(np.ldexp(a, -k))
+    return e4m3_encode(r), k, np.ldexp(r, k)
+
+
+def sampled_ce_e4m3(x, lm_head, targets, P, offset=0, stride=NEGATIVE_STRIDE, grad_loss=1.0,
+                    chunk=1024):
+    """Whole path with the logits GEMM on e4m3 operands (readings above)."""
+    lm_head = np.asarray(lm_head, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    V = lm_head.shape[0]
+    cand, tpos, vpos, info = build_candidates(targets, V, P, offset, stride)
+    w_c = gather_rows(lm_head, cand)
+    xq_codes, kx, xq = quantize_e4m3(x)
+    wq_codes, kw, wq = quantize_e4m3(w_c)
+    loss, lse, loss_rows, n = sampled_ce_forward(xq, wq, tpos, chunk)
+    dx, dW = sampled_ce_backward(grad_loss, x, w_c, cand, tpos, lse, V, chunk,
+                                 logit_x=xq, logit_w=wq)
+    return dict(candidates=cand, target_pos=tpos, vocab_pos=vpos, info=info, loss=loss,
+                lse=lse, loss_rows=loss_rows, n_valid=n, dx=dx, dW=dW,
+                x_codes=xq_codes, kx=kx, w_codes=wq_codes, kw=kw)
 
 
 # ---------------------------------------------------------------------------
