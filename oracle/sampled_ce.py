@@ -307,7 +307,7 @@ def sampled_ce(x, lm_head, targets, P, offset=0, stride=NEGATIVE_STRIDE, grad_lo
 #   * rounding: to nearest, ties to even, finite results saturate at +-448;
 #   * scale: one power of two per tensor (x, and W_C of the step): the
 #     smallest 2^k with amax * 2^-k <= 448, so scaling is exact and the codes
-#     are round(v * 2^-k); 2^0 for an all-zero tensor;
+#     are round(v * 2^-k); 2^0 for an all-zero tensor; k kept in [-126, 127];
 #   * only the logits GEMM uses them: z = (x_q 2^kx)(w_q 2^kw)^T; the softmax,
 #     loss and G follow from that z, and the gradient GEMMs use the bf16 x and
 #     W_C as in the bf16 path (the page does not give G's precision).
@@ -360,7 +360,9 @@ def e4m3_encode(r: np.ndarray) -> np.ndarray:
 
 
 def e4m3_scale_exponent(amax: float) -> int:
-    """The k of the per-tensor scale 2^k: smallest k with amax <= 448 * 2^k."""
+    """The k of the per-tensor scale 2^k: smallest k with amax <= 448 * 2^k,
+    kept in [-126, 127] so that 2^k and 2^-k are normal fp32 numbers (the
+    device scales by multiplying with them); 0 for an all-zero tensor."""
     amax = float(amax)
     if not amax > 0.0:
         return 0
@@ -370,7 +372,7 @@ def e4m3_scale_exponent(amax: float) -> int:
         k += 1
     while amax <= math.ldexp(E4M3_MAX, k - 1):
         k -= 1
-    return k
+    return min(max(k, -126), 127)
 
 
 def quantize_e4m3(a: np.ndarray):
@@ -410,21 +412,26 @@ def rows_forward(x_rows: np.ndarray, w_c: np.ndarray, tpos_rows: np.ndarray):
     return lse, loss_rows
 
 
-def dx_rows(x_rows, w_c, tpos_rows, lse_rows, scale):
-    """dX for a subset of rows: G_rows @ W_C."""
-    z = np.asarray(x_rows, dtype=np.float64) @ np.asarray(w_c, dtype=np.float64).T
+def dx_rows(x_rows, w_c, tpos_rows, lse_rows, scale, logit_x_rows=None, logit_w=None):
+    """dX for a subset of rows: G_rows @ W_C (G from logit_x_rows @ logit_w^T,
+    by default x_rows and W_C)."""
+    lx = x_rows if logit_x_rows is None else logit_x_rows
+    lw = w_c if logit_w is None else logit_w
+    z = np.asarray(lx, dtype=np.float64) @ np.asarray(lw, dtype=np.float64).T
     return dlogits(z, lse_rows, tpos_rows, scale) @ w_c
 
 
-def dw_c_rows(x, w_c, target_pos, lse, scale, cols, chunk=1024):
-    """dW_C[j] for j in ``cols`` only: sum_i G_ij x_i, over all rows."""
+def dw_c_rows(x, w_c, target_pos, lse, scale, cols, chunk=1024, logit_x=None, logit_w=None):
+    """dW_C[j] for j in ``cols`` only: sum_i G_ij x_i, over all rows (G from
+    logit_x @ logit_w^T, by default x and W_C)."""
     x = np.asarray(x, dtype=np.float64)
-    w_sel = np.asarray(w_c, dtype=np.float64)[cols]
+    lx = x if logit_x is None else np.asarray(logit_x, dtype=np.float64)
+    w_sel = np.asarray(w_c if logit_w is None else logit_w, dtype=np.float64)[cols]
     tpos = np.asarray(target_pos, dtype=np.int64)
     out = np.zeros((len(cols), x.shape[1]))
     col_of = {int(c): k for k, c in enumerate(cols)}
     for r0, r1 in _row_chunks(x.shape[0], chunk):
-        z = x[r0:r1] @ w_sel.T
+        z = lx[r0:r1] @ w_sel.T
         p = np.exp(z - lse[r0:r1, None])
         tp = tpos[r0:r1]
         for r in np.flatnonzero(tp >= 0):

@@ -78,6 +78,7 @@ def test_scale_exponent_definition():
     assert oc.e4m3_scale_exponent(np.nextafter(448.0, 1e9)) == 1
     assert oc.e4m3_scale_exponent(224.0) == -1
     assert oc.e4m3_scale_exponent(0.0) == 0
+    assert oc.e4m3_scale_exponent(1e-45) == -126  # clamped: 2^126 stays a normal fp32
     rng = np.random.default_rng(1)
     for amax in 10.0 ** rng.uniform(-30, 30, 200):
         k = oc.e4m3_scale_exponent(amax)
