@@ -156,6 +156,39 @@ SS_API ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const i
                         float* loss, float* lse, int32_t* n_valid, int32_t* dev_status,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* The forward above with the logits GEMM on 8-bit floating-point operands,
+ * as sampled_softmax.py keeps them (SampledLoss.rows: the candidate rows in
+ * float8 e4m3, fed to torch._scaled_mm). Format: OCP 8-bit floating point
+ * E4M3 (4 exponent bits, bias 7, 3 mantissa bits, largest finite 448).
+ * The pages give no scales; here each of x and W_C gets one power-of-two
+ * scale 2^k, the smallest with max|v| * 2^-k <= 448 (k in [-126, 127]), and
+ * the codes are v * 2^-k rounded to nearest even, saturating at +-448. The
+ * logits are z = 2^(kx + kw) (x_q . W_C,q) with fp32 accumulation on the
+ * tcgen05 tensor cores (kind::f8f6f4); lse, the loss and the gradient
+ * factors follow from that z exactly as in ss_ce_forward, so ss_ce_backward
+ * (bf16 gradient GEMMs on x and W_C) runs unchanged after it.
+ * Arguments as ss_ce_forward; additionally d % 16 == 0 and the workspace
+ * holds ss_workspace_bytes_e4m3(T, d, V, P) bytes (the bf16 layout plus the
+ * codes of x and W_C at its end). */
+SS_API ss_status ss_ce_forward_e4m3(const ss_bf16* x, const ss_bf16* lm_head,
+                                    const int32_t* candidates, const int32_t* target_pos,
+                                    int64_t T, int32_t d, int32_t V, int32_t P, float* loss,
+                                    float* lse, int32_t* n_valid, int32_t* dev_status,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes for ss_ce_forward_e4m3 (0 if the sizes are invalid or
+ * d % 16 != 0); it also serves the build and the backward. */
+SS_API size_t ss_workspace_bytes_e4m3(int64_t T, int32_t d, int32_t V, int32_t P);
+
+/* The per-tensor e4m3 quantization ss_ce_forward_e4m3 applies, on its own:
+ * dst[i] = code of src[i] * 2^-k (rounded to nearest even, saturating), with
+ * 2^k as above written to scale[0] (device float).
+ * In:  src [n] bf16, n % 8 == 0; scratch: 32 bytes of device memory (its
+ *      first 8 bytes are cleared by the call). All pointers 16-byte aligned.
+ * Out: dst [n] uint8 codes; scale [1] float32. */
+SS_API ss_status ss_quantize_e4m3(const ss_bf16* src, int64_t n, uint8_t* dst, float* scale,
+                                  void* scratch, void* stream);
+
 /* Backward of the loss above for an upstream gradient g = grad_loss[0]
  * ("Learning Triton ... Softmax", section "Gradient": softmax minus one-hot):
  *   G     = (g / n_valid) * (softmax - onehot)  (0 when n_valid = 0);

@@ -33,7 +33,7 @@ EXPORTS = (
     "ss_build_candidates_noalloc", "ss_ce_forward", "ss_ce_backward",
     "ss_status_string", "ss_last_cuda_error", "ss_version", "ss_timing_enable",
     "ss_timing_reset", "ss_timing_count", "ss_timing_query", "ss_prefix_positions",
-    "ss_selftest_wait_limit",
+    "ss_selftest_wait_limit", "ss_ce_forward_e4m3", "ss_workspace_bytes_e4m3", "ss_quantize_e4m3",
 )
 
 
@@ -76,6 +76,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ss_ce_backward": (_i32, [_p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _sz,
                                   _p]),
         "ss_prefix_positions": (_i32, [_p, _p, _p, _i64, _i32, _p, _p, _p]),
+        "ss_ce_forward_e4m3": (_i32, [_p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _p,
+                                      _sz, _p]),
+        "ss_workspace_bytes_e4m3": (_sz, [_i64, _i32, _i32, _i32]),
+        "ss_quantize_e4m3": (_i32, [_p, _i64, _p, _p, _p, _p]),
         "ss_selftest_wait_limit": (_i32, [_p, _p]),
         "ss_status_string": (ctypes.c_char_p, [_i32]),
         "ss_last_cuda_error": (ctypes.c_char_p, []),
@@ -162,6 +166,27 @@ def ss_ce_backward(grad_loss, candidates, vocab_pos, n_valid, T, d, V, P, dx, dW
     _check("ss_ce_backward", code)
 
 
+def ss_workspace_bytes_e4m3(T: int, d: int, V: int, P: int) -> int:
+    return int(load().ss_workspace_bytes_e4m3(T, d, V, P))
+
+
+def ss_ce_forward_e4m3(x, lm_head, candidates, target_pos, T, d, V, P, loss, lse, n_valid,
+                       dev_status, workspace, stream=None):
+    """ss_ce_forward with the logits GEMM on per-tensor e4m3 operands."""
+    code = load().ss_ce_forward_e4m3(
+        _ptr(x), _ptr(lm_head), _ptr(candidates), _ptr(target_pos), T, d, V, P, _ptr(loss),
+        _ptr(lse), _ptr(n_valid), _ptr(dev_status), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("ss_ce_forward_e4m3", code)
+
+
+def ss_quantize_e4m3(src, dst, scale, scratch, stream=None):
+    """dst = e4m3 codes of src * 2^-k; scale[0] = 2^k (per-tensor power of two)."""
+    code = load().ss_quantize_e4m3(_ptr(src), src.numel(), _ptr(dst), _ptr(scale), _ptr(scratch),
+                                   _stream(stream))
+    _check("ss_quantize_e4m3", code)
+
+
 def ss_prefix_positions(prefix_table, targets, vocab_pos, V, prefix_pos, dev_status, stream=None):
     """prefix_pos[i] = position in C of prefix_table[targets[i]], -1 if absent."""
     code = load().ss_prefix_positions(
@@ -218,10 +243,13 @@ class SampledCE:
     torch and calls the C ABI.
     """
 
-    def __init__(self, T: int, d: int, V: int, P: int, device="cuda"):
+    def __init__(self, T: int, d: int, V: int, P: int, device="cuda", precision: str = "bf16"):
+        if precision not in ("bf16", "e4m3"):
+            raise ValueError(f"precision {precision!r}: 'bf16' or 'e4m3' (logits GEMM operands)")
         self.T, self.d, self.V, self.P = T, d, V, P
+        self.precision = precision
         dev = torch.device(device)
-        ws = ss_workspace_bytes(T, d, V, P)
+        ws = (ss_workspace_bytes_e4m3 if precision == "e4m3" else ss_workspace_bytes)(T, d, V, P)
         if ws == 0:
             raise SampledCEError("ss_workspace_bytes", STATUS["SS_ERR_INVALID_ARG"],
                                  f"T={T} d={d} V={V} P={P}")
@@ -242,8 +270,9 @@ class SampledCE:
                             self.target_pos, self.vocab_pos, self.dev_status, self.workspace, stream)
 
     def forward(self, x, lm_head, stream=None):
-        ss_ce_forward(x, lm_head, self.candidates, self.target_pos, self.T, self.d, self.V, self.P,
-                      self.loss, self.lse, self.n_valid, self.dev_status, self.workspace, stream)
+        fwd = ss_ce_forward_e4m3 if self.precision == "e4m3" else ss_ce_forward
+        fwd(x, lm_head, self.candidates, self.target_pos, self.T, self.d, self.V, self.P,
+            self.loss, self.lse, self.n_valid, self.dev_status, self.workspace, stream)
 
     def backward(self, grad_loss=None, stream=None):
         g = self.grad_loss if grad_loss is None else grad_loss

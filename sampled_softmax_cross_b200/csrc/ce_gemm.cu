@@ -49,35 +49,58 @@ constexpr int A_STAGE = BM * BK * 2;   // 16 KB
 constexpr int B_STAGE = BNH * BK * 2;  // 16 KB
 constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
 constexpr int EPI_BUF = 32 * 64 * 2;  // one 32-row x 64-column bf16 box (4 KB)
-constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
 constexpr int BAR_BYTES = 256;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr int NUM_THREADS = 192;
 constexpr float LOG2E = 1.4426950408889634f;
 
-// Stages: as many as shared memory allows. The forward's E is a 2.4 GB write
-// stream, which TMA bulk stores from a staging box handle far better than
-// 16-byte stores from registers (1.47 vs 1.89 ms measured); the box costs
-// one stage. dX and dW store little and use the 7th stage instead.
+// Per kind: operand majors, the E store path, pipeline stages and epilogue
+// warps. The forward stores the 2.4 GB E stream through staging boxes and
+// TMA bulk stores (1.47 ms against 1.89 ms with 16-byte register stores,
+// measured); the boxes cost one operand stage. With e4m3 operands the MMAs
+// of a tile take half as long (6 K blocks of 128 at twice the rate), and the
+// epilogue -- TMEM loads, an exponential per element, packing, staging and
+// stores -- becomes the longer part: that kind gets two warps per TMEM lane
+// quarter, each taking half of the tile's columns (8% faster measured; the
+// bf16 forward gains nothing from it). dX and dW (hundreds of K blocks per
+// tile) store little, from registers, and use a 7th stage.
 template <int KIND>
 struct Op;
 template <>
 struct Op<KIND_FWD> {  // A = x (K-major), B = W_C (K-major)
-  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6;
+  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6, EPI_WARPS = 4;
+};
+template <>
+struct Op<KIND_FWD8> {  // A = x_q, B = W_C,q (e4m3, K-major; 128 per K block)
+  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 5, EPI_WARPS = 8;
 };
 template <>
 struct Op<KIND_DX> {  // A = E' (K-major), B = W_C viewed [K=P][N=d] (MN-major)
-  static constexpr int A_MN = 0, B_MN = 1, TMA_STORE = 0, STAGES = 7;
+  static constexpr int A_MN = 0, B_MN = 1, TMA_STORE = 0, STAGES = 7, EPI_WARPS = 4;
 };
 template <>
 struct Op<KIND_DW> {  // A = E' viewed [K=T][M=P] (MN-major), B = x' viewed [K=T][N=d] (MN-major)
-  static constexpr int A_MN = 1, B_MN = 1, TMA_STORE = 0, STAGES = 7;
+  static constexpr int A_MN = 1, B_MN = 1, TMA_STORE = 0, STAGES = 7, EPI_WARPS = 4;
 };
+
+static_assert(Op<KIND_FWD>::EPI_WARPS / 4 == kFwdSumsPerTileBf16 &&
+                  Op<KIND_FWD8>::EPI_WARPS / 4 == kFwdSumsPerTileE4m3,
+              "row sums per tile");
+
+// warp 0 producer, warp 1 TMEM owner / MMA issuer, then the epilogue warps
+template <int KIND>
+constexpr int num_threads() {
+  return 64 + 32 * Op<KIND>::EPI_WARPS;
+}
+template <int KIND>
+constexpr int epi_bytes() {
+  return Op<KIND>::TMA_STORE ? Op<KIND>::EPI_WARPS * 2 * EPI_BUF : 0;
+}
 template <int KIND>
 constexpr int smem_bytes() {
-  return 1024 + Op<KIND>::STAGES * STAGE_BYTES + (Op<KIND>::TMA_STORE ? EPI_BYTES : 0) + BAR_BYTES;
+  return 1024 + Op<KIND>::STAGES * STAGE_BYTES + epi_bytes<KIND>() + BAR_BYTES;
 }
-static_assert(smem_bytes<KIND_FWD>() <= 232448 && smem_bytes<KIND_DX>() <= 232448 &&
+static_assert(smem_bytes<KIND_FWD>() <= 232448 && smem_bytes<KIND_FWD8>() <= 232448 &&
+                  smem_bytes<KIND_DX>() <= 232448 &&
                   smem_bytes<KIND_DW>() <= 232448,
               "shared memory budget");
 
@@ -136,16 +159,18 @@ cudaError_t launch_wait_selftest(int32_t* status, cudaStream_t s) {
 }
 
 template <int KIND>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(), 1)
     k_gemm(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
            const __grid_constant__ CUtensorMap tma_c, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   constexpr int STAGES = Op<KIND>::STAGES;
+  constexpr bool IS_FWD = KIND == KIND_FWD || KIND == KIND_FWD8;
+  constexpr bool F8 = KIND == KIND_FWD8;
+  constexpr int BKE = F8 ? 2 * BK : BK;  // K elements per 128-byte row of a stage
   uint8_t* epi_smem = smem + STAGES * STAGE_BYTES;
-  uint64_t* full =
-      reinterpret_cast<uint64_t*>(epi_smem + (Op<KIND>::TMA_STORE ? EPI_BYTES : 0));
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + epi_bytes<KIND>());
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -164,7 +189,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);   // one multicast commit per finished accumulator
-      mbar_init(&tempty[a], 8);  // leader: 4 epilogue warps of each CTA
+      mbar_init(&tempty[a], 2 * Op<KIND>::EPI_WARPS);  // leader: epilogue warps of both CTAs
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -200,7 +225,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
           uint8_t* sa = smem + stage * STAGE_BYTES;
           uint8_t* sb = sa + A_STAGE;
-          const int k0 = kb * BK;
+          const int k0 = kb * BKE;
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
           if (Op<KIND>::A_MN) {
@@ -235,7 +260,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------- MMA issuer (leader only) --
     if (rank == 0) {
-      constexpr uint32_t IDESC = idesc_bf16(2 * BM, BN, Op<KIND>::A_MN, Op<KIND>::B_MN);
+      constexpr uint32_t IDESC =
+          F8 ? idesc_e4m3(2 * BM, BN) : idesc_bf16(2 * BM, BN, Op<KIND>::A_MN, Op<KIND>::B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -261,7 +287,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                                                  : sdesc_sw128(a_addr + kk * 32, 16, 1024);
               const uint64_t bd = Op<KIND>::B_MN ? sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
                                                  : sdesc_sw128(b_addr + kk * 32, 16, 1024);
-              umma_bf16_pair(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+              if (F8)  // K = 32 e4m3 per MMA: the same 32 bytes as 16 bf16
+                umma_f8_pair(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+              else
+                umma_bf16_pair(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
             }
             umma_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
           }
@@ -278,14 +307,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ----------------------------------------------------------- epilogue --
+    constexpr int EW = Op<KIND>::EPI_WARPS;
+    constexpr int HALVES = EW / 4;        // warps per TMEM lane quarter
+    constexpr int CPW = BN / 64 / HALVES;  // 64-column chunks per warp and tile
     const int q = warp & 3;   // TMEM lane quarter this warp may access
     const int e = warp - 2;   // staging slot
+    const int half = e / 4;   // which part of the tile's columns
+    const int c_begin = half * CPW;
     int it = 0;
     uint32_t store_ctr = 0;
     // the forward's E is a write-once stream larger than L2: evict it first
-    const uint64_t store_policy = KIND == KIND_FWD ? policy_evict_first() : 0;
+    const uint64_t store_policy = IS_FWD ? policy_evict_first() : 0;
+    // forward: log2(e) times the logits' scale (the operand scales for e4m3)
+    const float zs = F8 ? LOG2E * __ldg(args.qscale + 2) : LOG2E;
     float scale = 1.f;  // dX / dW: g / n (0 when no row is valid)
-    if (KIND != KIND_FWD) {
+    if (!IS_FWD) {
       const int nv = __ldg(args.n_valid);
       scale = nv > 0 ? __ldg(args.grad_loss) / (float)nv : 0.f;
     }
@@ -294,7 +330,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       // write them while the first tiles' MMAs run (they are disjoint from
       // the rows the tiles scatter). Each warp takes blocks of 32 classes.
       const int vpr = args.N / 8;
-      const int64_t gw = (int64_t)blockIdx.x * 4 + e, nw = (int64_t)gridDim.x * 4;
+      const int64_t gw = (int64_t)blockIdx.x * EW + e, nw = (int64_t)gridDim.x * EW;
       uint4* dW4 = reinterpret_cast<uint4*>(args.dW);
       for (int64_t base = gw * 32; base < args.V; base += nw * 32) {
         const int64_t r = base + lane;
@@ -321,7 +357,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       bool keep = true;  // forward: store E (false on ignored rows: store 0)
       float rs = scale;  // dX: (g / n) * r_i
       int32_t cls = -1;
-      if (KIND == KIND_FWD && row_ok) {
+      if (IS_FWD && row_ok) {
         ref2 = __ldg(args.ref + row) * LOG2E;
         keep = __ldg(args.tpos + row) >= 0;
       }
@@ -332,16 +368,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
 
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const int n_chunks = min(BN / 64, (args.N - n0 + 63) / 64);
+      const int n_chunks = min(BN / 64, (args.N - n0 + 63) / 64);  // with valid columns
+      const int c_end = min(c_begin + CPW, n_chunks);
       float s_tile = 0.f;
+      if (c_begin >= c_end) {  // no valid column of this tile for this warp
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+      }
 
-      for (int c = 0; c < n_chunks; ++c) {
+      for (int c = c_begin; c < c_end; ++c) {
         const int col0 = n0 + c * 64;
         uint32_t r0[32], r1[32];
         tmem_ld32(t_row + c * 64, r0);
         tmem_ld32(t_row + c * 64 + 32, r1);
         tmem_wait_ld();
-        if (c == n_chunks - 1) {
+        if (c == c_end - 1) {
           // all TMEM reads of this accumulator are done: hand it back to the leader
           tc_fence_before();
           __syncwarp();
@@ -354,7 +396,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           v[32 + j] = __uint_as_float(r1[j]);
         }
 
-        if (KIND == KIND_FWD) {
+        if (IS_FWD) {
           // E = exp(z - ref) and its row sum over the tile's valid columns
           const int nvalid = min(64, args.N - col0);
           float sp[8];  // independent partial sums (short dependency chains)
@@ -363,13 +405,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           if (nvalid == 64) {
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
-              v[j] = ex2_approx(fmaf(v[j], LOG2E, -ref2));
+              v[j] = ex2_approx(fmaf(v[j], zs, -ref2));
               sp[j & 7] += v[j];
             }
           } else {
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
-              v[j] = j < nvalid ? ex2_approx(fmaf(v[j], LOG2E, -ref2)) : 0.f;
+              v[j] = j < nvalid ? ex2_approx(fmaf(v[j], zs, -ref2)) : 0.f;
               sp[j & 7] += v[j];
             }
           }
@@ -402,7 +444,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           fence_async_smem();
           __syncwarp();
           if (lane == 0 && m0 + q * 32 < args.M) {
-            if (KIND == KIND_FWD)
+            if (IS_FWD)
               tma_store_2d_hint(&tma_c, buf, col0, m0 + q * 32, store_policy);
             else
               tma_store_2d(&tma_c, buf, col0, m0 + q * 32);
@@ -420,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                                            pack_bf16x2(v[cc * 8 + 2], v[cc * 8 + 3]),
                                            pack_bf16x2(v[cc * 8 + 4], v[cc * 8 + 5]),
                                            pack_bf16x2(v[cc * 8 + 6], v[cc * 8 + 7]));
-                if (KIND == KIND_FWD)
+                if (IS_FWD)
                   __stcs(dst + cc, w);  // E is a write-once stream: do not keep it in L2
                 else
                   dst[cc] = w;
@@ -445,7 +487,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
       }
 
-      if (KIND == KIND_FWD && row_ok) args.rowsum[(size_t)n_blk * args.M + row] = s_tile;
+      if (IS_FWD && row_ok) args.rowsum[(size_t)(n_blk * HALVES + half) * args.M + row] = s_tile;
     }
     if (lane == 0) bulk_wait<0>();
     __syncwarp();
@@ -471,6 +513,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 int gemm_smem_bytes(int kind) {
   switch (kind) {
     case KIND_FWD: return smem_bytes<KIND_FWD>();
+    case KIND_FWD8: return smem_bytes<KIND_FWD8>();
     case KIND_DX: return smem_bytes<KIND_DX>();
     default: return smem_bytes<KIND_DW>();
   }
@@ -479,16 +522,26 @@ int gemm_smem_bytes(int kind) {
 const void* gemm_kernel_ptr(int kind) {
   switch (kind) {
     case KIND_FWD: return reinterpret_cast<const void*>(&k_gemm<KIND_FWD>);
+    case KIND_FWD8: return reinterpret_cast<const void*>(&k_gemm<KIND_FWD8>);
     case KIND_DX: return reinterpret_cast<const void*>(&k_gemm<KIND_DX>);
     default: return reinterpret_cast<const void*>(&k_gemm<KIND_DW>);
   }
 }
 
 // How many CTA pairs of this kernel can be resident at once on the device.
+int gemm_threads(int kind) {
+  switch (kind) {
+    case KIND_FWD: return num_threads<KIND_FWD>();
+    case KIND_FWD8: return num_threads<KIND_FWD8>();
+    case KIND_DX: return num_threads<KIND_DX>();
+    default: return num_threads<KIND_DW>();
+  }
+}
+
 int gemm_max_pairs(int kind, int sms) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (sms / 2));
-  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.blockDim = dim3(gemm_threads(kind));
   cfg.dynamicSmemBytes = gemm_smem_bytes(kind);
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
@@ -507,9 +560,10 @@ int gemm_max_pairs(int kind, int sms) {
 
 cudaError_t launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                         const GemmArgs& args, int pairs, cudaStream_t s) {
-  dim3 g(2 * pairs), blk(NUM_THREADS);
+  dim3 g(2 * pairs), blk(gemm_threads(kind));
   switch (kind) {
     case KIND_FWD: k_gemm<KIND_FWD><<<g, blk, smem_bytes<KIND_FWD>(), s>>>(a, b, c, args); break;
+    case KIND_FWD8: k_gemm<KIND_FWD8><<<g, blk, smem_bytes<KIND_FWD8>(), s>>>(a, b, c, args); break;
     case KIND_DX: k_gemm<KIND_DX><<<g, blk, smem_bytes<KIND_DX>(), s>>>(a, b, c, args); break;
     default: k_gemm<KIND_DW><<<g, blk, smem_bytes<KIND_DW>(), s>>>(a, b, c, args); break;
   }

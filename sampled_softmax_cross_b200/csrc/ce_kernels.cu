@@ -5,12 +5,16 @@
 // lm_head gradient.
 #include <limits.h>
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "sm100.cuh"
 #include "ss_internal.h"
 
 namespace ssb {
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 constexpr int kBuildThreads = 1024;
 
 // ----------------------------------------------------------------------------
@@ -347,6 +351,154 @@ __global__ void k_ref_logits(const uint4* __restrict__ x, const uint4* __restric
 }
 
 // ----------------------------------------------------------------------------
+// e4m3 (OCP 8-bit floating point, E4M3) helpers. Codes are produced by the
+// hardware conversion (round to nearest even, saturating at +-448) and read
+// back through fp16, which holds every e4m3 value exactly.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two_codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(two_codes, __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+__device__ __forceinline__ uint16_t float2_to_e4m3x2(float lo, float hi) {
+  return __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
+
+// Exponent k of the per-tensor scale: the smallest k with amax <= 448 * 2^k,
+// kept in [-126, 127] (2^k and 2^-k normal); 0 for an all-zero tensor.
+__device__ __forceinline__ int e4m3_scale_exp(float amax) {
+  if (!(amax > 0.f)) return 0;
+  int ex;
+  frexpf(amax, &ex);
+  int k = ex - 9;
+  for (int i = 0; i < 4 && amax > ldexpf(448.f, k); ++i) ++k;
+  for (int i = 0; i < 4 && amax <= ldexpf(448.f, k - 1); ++i) --k;
+  return min(max(k, -126), 127);
+}
+
+// amax[0] = max |a|, amax[1] = max |b| as bf16 bit patterns (monotonic in
+// the magnitude for finite values), by atomicMax.
+__global__ void k_amax_bf16(const uint4* __restrict__ a, int64_t na, const uint4* __restrict__ b,
+                            int64_t nb, uint32_t* __restrict__ amax) {
+  uint32_t ma = 0, mb = 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  constexpr int U = 4;  // independent loads in flight per thread
+  for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < na + nb;
+       i0 += U * stride) {
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u * stride;
+      v[u] = i < na ? __ldg(a + i) : (i < na + nb ? __ldg(b + (i - na)) : make_uint4(0, 0, 0, 0));
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint32_t m = 0;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) m = max(m, max(w[h] & 0x7fffu, (w[h] >> 16) & 0x7fffu));
+      if (i0 + u * stride < na)
+        ma = max(ma, m);
+      else
+        mb = max(mb, m);
+    }
+  }
+  // one atomic per block and tensor: per-warp atomics on one address serialise
+  __shared__ uint32_t s_m[2][32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, o));
+    mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+  }
+  if ((threadIdx.x & 31) == 0) {
+    s_m[0][threadIdx.x >> 5] = ma;
+    s_m[1][threadIdx.x >> 5] = mb;
+  }
+  __syncthreads();
+  if (threadIdx.x < 2) {
+    uint32_t m = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = max(m, s_m[threadIdx.x][w]);
+    if (m) atomicMax(amax + threadIdx.x, m);
+  }
+}
+
+__global__ void k_quant_e4m3(const uint4* __restrict__ a, int64_t na, uint2* __restrict__ a8,
+                             const uint4* __restrict__ b, int64_t nb, uint2* __restrict__ b8,
+                             const uint32_t* __restrict__ amax, float* __restrict__ qscale) {
+  const int ka = e4m3_scale_exp(__uint_as_float(amax[0] << 16));
+  const int kb = e4m3_scale_exp(__uint_as_float(amax[1] << 16));
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    qscale[0] = ldexpf(1.f, ka);
+    qscale[1] = ldexpf(1.f, kb);
+    qscale[2] = ldexpf(1.f, ka + kb);
+  }
+  const float ia = ldexpf(1.f, -ka), ib = ldexpf(1.f, -kb);  // exact: powers of two
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  constexpr int U = 4;  // independent loads in flight per thread
+  for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < na + nb;
+       i0 += U * stride) {
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u * stride;
+      v[u] = i < na ? __ldg(a + i) : (i < na + nb ? __ldg(b + (i - na)) : make_uint4(0, 0, 0, 0));
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i >= na + nb) break;
+      const bool in_a = i < na;
+      const float sc = in_a ? ia : ib;
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint16_t q[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        q[h] = float2_to_e4m3x2(__uint_as_float(w[h] << 16) * sc,
+                                __uint_as_float(w[h] & 0xffff0000u) * sc);
+      const uint2 out = make_uint2((uint32_t)q[0] | ((uint32_t)q[1] << 16),
+                                   (uint32_t)q[2] | ((uint32_t)q[3] << 16));
+      if (in_a)
+        a8[i] = out;
+      else
+        b8[i - na] = out;
+    }
+  }
+}
+
+// Reference logit for the e4m3 forward: the same dot product the GEMM forms
+// (codes times the product of the two scales), fp32. One warp per row.
+__global__ void k_ref_logits_e4m3(const uint4* __restrict__ x8, const uint4* __restrict__ w8,
+                                  const int32_t* __restrict__ tpos, int64_t T, int32_t vpr,
+                                  int32_t P, const float* __restrict__ qscale,
+                                  float* __restrict__ ref) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const float s = __ldg(qscale + 2);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < T; r += warps) {
+    const int t = __ldg(tpos + r);
+    const int j = (t >= 0 && t < P) ? t : 0;
+    float acc = 0.f;
+    for (int v = lane; v < vpr; v += 32) {
+      const uint4 xa = __ldg(x8 + r * vpr + v), wa = __ldg(w8 + (int64_t)j * vpr + v);
+      const uint32_t xw[4] = {xa.x, xa.y, xa.z, xa.w}, ww[4] = {wa.x, wa.y, wa.z, wa.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 x0 = e4m3x2_to_float2((uint16_t)(xw[h] & 0xffffu));
+        const float2 x1 = e4m3x2_to_float2((uint16_t)(xw[h] >> 16));
+        const float2 w0 = e4m3x2_to_float2((uint16_t)(ww[h] & 0xffffu));
+        const float2 w1 = e4m3x2_to_float2((uint16_t)(ww[h] >> 16));
+        acc = fmaf(x0.x, w0.x, acc);
+        acc = fmaf(x0.y, w0.y, acc);
+        acc = fmaf(x1.x, w1.x, acc);
+        acc = fmaf(x1.y, w1.y, acc);
+      }
+    }
+    const float sum = warp_sum(acc);
+    if (lane == 0) ref[r] = sum * s;
+  }
+}
+
+// ----------------------------------------------------------------------------
 // Row pass after the forward GEMM. With S_i = sum of the row's per-tile sums of
 // exp(z - ref_i):
 //   lse_i = ref_i + log S_i,   loss_i = lse_i - z_target = log S_i (valid rows),
@@ -389,7 +541,7 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a) {
     const bool in = r < a.T;
     float s = 0.f;
     if (in)
-      for (int t = lane >> 3; t < a.tiles_n; t += 4) s += __ldg(a.rowsum + (int64_t)t * a.T + r);
+      for (int t = lane >> 3; t < a.nsums; t += 4) s += __ldg(a.rowsum + (int64_t)t * a.T + r);
     s += __shfl_xor_sync(0xffffffffu, s, 8);
     s += __shfl_xor_sync(0xffffffffu, s, 16);
     const float S = s;  // identical in the four lanes of the row
@@ -494,6 +646,22 @@ __device__ __forceinline__ float row_logit(const uint4* xr, const uint4* wr, int
   return acc;
 }
 
+// Logit of row r and class j in the row pass's precision: bf16 x . W_C, or
+// for the e4m3 forward, the scales times the dot product of the codes.
+__device__ __forceinline__ float row_logit_any(const RowArgs& a, int64_t r, int64_t j, int vpr) {
+  if (a.x8 == nullptr)
+    return row_logit(reinterpret_cast<const uint4*>(a.x) + r * vpr,
+                     reinterpret_cast<const uint4*>(a.w_c) + j * vpr, vpr);
+  float acc = 0.f;
+  for (int k = 0; k < a.d; k += 2) {
+    const float2 xf = e4m3x2_to_float2(*reinterpret_cast<const uint16_t*>(a.x8 + r * a.d + k));
+    const float2 wf = e4m3x2_to_float2(*reinterpret_cast<const uint16_t*>(a.w8 + j * a.d + k));
+    acc = fmaf(xf.x, wf.x, acc);
+    acc = fmaf(xf.y, wf.y, acc);
+  }
+  return acc * __ldg(a.qscale + 2);
+}
+
 __global__ void __launch_bounds__(kFinThreads) k_finalize(RowArgs a, int32_t nparts) {
   __shared__ float sh[33];
   __shared__ float s_zt;
@@ -506,14 +674,13 @@ __global__ void __launch_bounds__(kFinThreads) k_finalize(RowArgs a, int32_t npa
     const int tp = a.tpos[r];
     const bool valid = tp >= 0 && tp < a.P;
     const uint4* xr = reinterpret_cast<const uint4*>(a.x) + r * vpr;
-    const uint4* w = reinterpret_cast<const uint4*>(a.w_c);
     float m = -INFINITY;
-    for (int j = threadIdx.x; j < a.P; j += nt) m = fmaxf(m, row_logit(xr, w + (int64_t)j * vpr, vpr));
+    for (int j = threadIdx.x; j < a.P; j += nt) m = fmaxf(m, row_logit_any(a, r, j, vpr));
     m = block_reduce(m, true, sh);
     float sum = 0.f;
     uint16_t* ur = a.u + r * a.ldz;
     for (int j = threadIdx.x; j < a.P; j += nt) {
-      const float z = row_logit(xr, w + (int64_t)j * vpr, vpr);
+      const float z = row_logit_any(a, r, j, vpr);
       const float e = expf(z - m);
       sum += e;
       ur[j] = valid ? (uint16_t)(pack_bf16x2(e, 0.f) & 0xffffu) : (uint16_t)0;
@@ -714,6 +881,39 @@ cudaError_t launch_prefix_pos(const int32_t* prefix_table, const int32_t* target
   if (T == 0) return cudaSuccess;
   const int blocks = (int)min64((T + 255) / 256, (int64_t)num_sms() * 8);
   k_prefix_pos<<<blocks, 256, 0, s>>>(prefix_table, targets, vocab_pos, T, V, prefix_pos, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_amax_bf16(const uint16_t* a, int64_t n, const uint16_t* b, int64_t m,
+                             uint32_t* amax, cudaStream_t s) {
+  const int64_t vec = (n + m) / 8;
+  if (vec == 0) return cudaSuccess;
+  const int blocks = (int)min64((vec + 255) / 256, (int64_t)num_sms() * 8);
+  k_amax_bf16<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(a), n / 8,
+                                     reinterpret_cast<const uint4*>(b), m / 8, amax);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_e4m3(const uint16_t* a, int64_t n, uint8_t* a8, const uint16_t* b,
+                              int64_t m, uint8_t* b8, const uint32_t* amax, float* qscale,
+                              cudaStream_t s) {
+  const int64_t vec = (n + m) / 8;
+  const int blocks = (int)max64(1, min64((vec + 255) / 256, (int64_t)num_sms() * 8));
+  k_quant_e4m3<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(a), n / 8,
+                                      reinterpret_cast<uint2*>(a8),
+                                      reinterpret_cast<const uint4*>(b), m / 8,
+                                      reinterpret_cast<uint2*>(b8), amax, qscale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ref_logits_e4m3(const uint8_t* x8, const uint8_t* w8, const int32_t* tpos,
+                                   int64_t T, int32_t d, int32_t P, const float* qscale,
+                                   float* ref, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = (int)min64((T + 7) / 8, (int64_t)num_sms() * 16);
+  k_ref_logits_e4m3<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(x8),
+                                           reinterpret_cast<const uint4*>(w8), tpos, T, d / 16, P,
+                                           qscale, ref);
   return cudaGetLastError();
 }
 

@@ -319,6 +319,18 @@ SS_DEV void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint
       : "memory");
 }
 
+// Same MMA on 8-bit floating-point operands (kind::f8f6f4; the formats are in
+// the instruction descriptor), fp32 accumulation.
+SS_DEV void umma_f8_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on the mbarrier at this shared-memory offset in every CTA of
 // `cta_mask` once the MMAs issued so far by this thread have completed.
 SS_DEV void umma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
@@ -370,6 +382,16 @@ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
          | ((uint32_t)b_mn_major << 16)     // B major (0 = K)
          | ((uint32_t)(N >> 3) << 17)       // N / 8
          | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+// Instruction descriptor: e4m3 x e4m3 -> fp32 (kind::f8f6f4, format code 0
+// for both operands), dense, M x N, both operands K-major.
+constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4)                      // D format: f32
+         | (0u << 7)                    // A format: e4m3
+         | (0u << 10)                   // B format: e4m3
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
 // ------------------------------------------------------------------ misc --

@@ -31,7 +31,7 @@ ss_status cuda_fail(cudaError_t e, const char* where) {
 struct DeviceState {
   bool ready = false;
   int sms = 0;
-  int max_pairs[3] = {0, 0, 0};  // resident CTA pairs of each GEMM kernel
+  int max_pairs[kNumGemmKinds] = {};  // resident CTA pairs of each GEMM kernel
   ss_status status = SS_OK;
 };
 std::mutex g_dev_mu;
@@ -52,7 +52,7 @@ ss_status ensure_device(int* sms, int* max_pairs = nullptr) {
     if (major != 10) {
       d.status = SS_ERR_UNSUPPORTED_DEVICE;
     } else {
-      for (int k = 0; k < 3; ++k) {
+      for (int k = 0; k < kNumGemmKinds; ++k) {
         SS_CUDA(cudaFuncSetAttribute(gemm_kernel_ptr(k),
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      gemm_smem_bytes(k)),
@@ -64,7 +64,7 @@ ss_status ensure_device(int* sms, int* max_pairs = nullptr) {
   }
   *sms = d.sms;
   if (max_pairs != nullptr)
-    for (int k = 0; k < 3; ++k) max_pairs[k] = d.max_pairs[k];
+    for (int k = 0; k < kNumGemmKinds; ++k) max_pairs[k] = d.max_pairs[k];
   return d.status;
 }
 
@@ -83,19 +83,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer][inner] with row pitch `row_elems`, 128-byte swizzle.
+// 2-D tensor [outer][inner] of bf16 (or, with elem_bytes 1, e4m3 codes) with
+// row pitch `row_elems`, 128-byte swizzle.
 ss_status make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
-                   uint64_t row_elems, uint32_t box_inner, uint32_t box_outer) {
+                   uint64_t row_elems, uint32_t box_inner, uint32_t box_outer,
+                   int elem_bytes = 2) {
   auto fn = encode_fn();
   if (fn == nullptr) {
     snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
     return SS_ERR_CUDA;
   }
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_elems * 2};
+  cuuint64_t strides[1] = {row_elems * (uint64_t)elem_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+  CUresult r = fn(m, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  2, const_cast<void*>(ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -155,6 +158,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 struct Layout {
   size_t bitmap, prefix, ref, rscale, loss_rows, fix_list, fix_count, partials, w_c, u, rowsum, xs,
       total;
+  size_t x8, w8, qscale, total_e4m3;  // after `total`: the e4m3 forward's extra buffers
   int64_t ldz;
   int tiles_n;
 };
@@ -186,9 +190,14 @@ Layout layout(int64_t T, int32_t d, int32_t V, int32_t P) {
   L.partials = take((size_t)kRowPartials * sizeof(double2), 256);
   L.w_c = take((size_t)P * d * 2, 1024);
   L.u = take((size_t)T * L.ldz * 2, 1024);
-  L.rowsum = take((size_t)L.tiles_n * T * 4, 1024);
+  L.rowsum = take((size_t)L.tiles_n * kFwdSumsPerTileE4m3 * T * 4, 1024);  // the larger count
   L.xs = take((size_t)T * d * 2, 1024);
   L.total = align_up(off, 1024);
+  off = L.total;
+  L.x8 = take((size_t)T * d, 1024);
+  L.w8 = take((size_t)P * d, 1024);
+  L.qscale = take(16, 256);
+  L.total_e4m3 = align_up(off, 1024);
   return L;
 }
 
@@ -206,6 +215,109 @@ int gcd_int(int64_t a, int64_t b) {
 }  // namespace
 
 // ===================================================================== API ==
+// The forward, with the logits GEMM on bf16 operands or (e4m3) on per-tensor
+// e4m3 quantizations of x and W_C.
+static ss_status forward_impl(const ss_bf16* x, const ss_bf16* lm_head,
+                              const int32_t* candidates, const int32_t* target_pos, int64_t T,
+                              int32_t d, int32_t V, int32_t P, float* loss, float* lse,
+                              int32_t* n_valid, int32_t* dev_status, void* workspace,
+                              size_t workspace_bytes, void* stream, bool e4m3) {
+  if (!sizes_ok(T, d, V, P) || (e4m3 && d % 16 != 0)) return SS_ERR_INVALID_ARG;
+  if (lm_head == nullptr || candidates == nullptr || loss == nullptr || n_valid == nullptr ||
+      dev_status == nullptr || workspace == nullptr ||
+      (T > 0 && (x == nullptr || target_pos == nullptr || lse == nullptr)))
+    return SS_ERR_INVALID_ARG;
+  if (!aligned16(lm_head) || !aligned16(workspace) || (T > 0 && !aligned16(x)))
+    return SS_ERR_MISALIGNED;
+  const Layout L = layout(T, d, V, P);
+  if (workspace_bytes < (e4m3 ? L.total_e4m3 : L.total)) return SS_ERR_WORKSPACE_TOO_SMALL;
+  int sms, pairs[kNumGemmKinds];
+  ss_status ds = ensure_device(&sms, pairs);
+  if (ds != SS_OK) return ds;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* w_c = reinterpret_cast<uint16_t*>(ws + L.w_c);
+  uint16_t* u = reinterpret_cast<uint16_t*>(ws + L.u);
+  float* ref = reinterpret_cast<float*>(ws + L.ref);
+  float* rowsum = reinterpret_cast<float*>(ws + L.rowsum);
+  float* loss_rows = reinterpret_cast<float*>(ws + L.loss_rows);
+  int32_t* fix_count = reinterpret_cast<int32_t*>(ws + L.fix_count);
+  int32_t* kstatus = dev_status + 8;
+
+  RowArgs ra{};
+  ra.rowsum = rowsum;
+  ra.ref = ref;
+  ra.tpos = target_pos;
+  ra.x = x;
+  ra.T = T;
+  ra.d = d;
+  ra.P = P;
+  ra.nsums = L.tiles_n * (e4m3 ? kFwdSumsPerTileE4m3 : kFwdSumsPerTileBf16);
+  ra.ldz = L.ldz;
+  ra.w_c = w_c;
+  ra.u = u;
+  ra.lse = lse;
+  ra.rscale = reinterpret_cast<float*>(ws + L.rscale);
+  ra.xs = reinterpret_cast<uint16_t*>(ws + L.xs);
+  ra.loss_rows = loss_rows;
+  ra.fix_list = reinterpret_cast<int32_t*>(ws + L.fix_list);
+  ra.fix_count = fix_count;
+  ra.partials = reinterpret_cast<double2*>(ws + L.partials);
+  ra.loss = loss;
+  ra.n_valid = n_valid;
+  uint8_t* x8 = ws + L.x8;
+  uint8_t* w8 = ws + L.w8;
+  float* qscale = reinterpret_cast<float*>(ws + L.qscale);
+  uint32_t* amax = reinterpret_cast<uint32_t*>(fix_count + 1);  // zeroed with fix_count
+  if (e4m3) {
+    ra.x8 = x8;
+    ra.w8 = w8;
+    ra.qscale = qscale;
+  }
+
+  SS_LAUNCH("gather", s,
+            launch_gather(lm_head, candidates, P, d, V, w_c, kstatus, fix_count, e4m3 ? 3 : 1, s));
+  if (T > 0) {
+    CUtensorMap ta, tb, tc;
+    ss_status r;
+    if (e4m3) {
+      SS_LAUNCH("amax_e4m3", s, launch_amax_bf16(x, T * d, w_c, (int64_t)P * d, amax, s));
+      SS_LAUNCH("quant_e4m3", s,
+                launch_quant_e4m3(x, T * d, x8, w_c, (int64_t)P * d, w8, amax, qscale, s));
+      SS_LAUNCH("ref_logits_e4m3", s,
+                launch_ref_logits_e4m3(x8, w8, target_pos, T, d, P, qscale, ref, s));
+      if ((r = make_map(&ta, x8, d, T, d, 128, kBM, 1)) != SS_OK) return r;
+      if ((r = make_map(&tb, w8, d, P, d, 128, kBN / 2, 1)) != SS_OK) return r;
+    } else {
+      SS_LAUNCH("ref_logits", s, launch_ref_logits(x, w_c, target_pos, T, d, P, ref, s));
+      if ((r = make_map(&ta, x, d, T, d, 64, kBM)) != SS_OK) return r;
+      if ((r = make_map(&tb, w_c, d, P, d, 64, kBN / 2)) != SS_OK) return r;
+    }
+    if ((r = make_map(&tc, u, P, T, L.ldz, 64, 32)) != SS_OK) return r;
+    GemmArgs a{};
+    a.M = (int32_t)T;
+    a.N = P;
+    a.K = d;
+    a.tiles_m = (int32_t)((T + kBMP - 1) / kBMP);
+    a.tiles_n = L.tiles_n;
+    a.num_kb = e4m3 ? (d + 127) / 128 : (d + 63) / 64;
+    a.tpos = target_pos;
+    a.ref = ref;
+    a.qscale = e4m3 ? qscale : nullptr;
+    a.rowsum = rowsum;
+    a.out = u;
+    a.ld_out = L.ldz;
+    a.status = kstatus;
+    const int tiles = a.tiles_m * a.tiles_n;
+    const int kind = e4m3 ? KIND_FWD8 : KIND_FWD;
+    SS_LAUNCH(e4m3 ? "fwd_gemm_ce_e4m3" : "fwd_gemm_ce", s,
+              launch_gemm(kind, ta, tb, tc, a, tiles < pairs[kind] ? tiles : pairs[kind], s));
+    SS_LAUNCH("row_pass", s, launch_rows(ra, s));
+  }
+  SS_LAUNCH("loss_finalize", s, launch_finalize(ra, s));
+  return SS_OK;
+}
+
 extern "C" {
 
 int32_t ss_version(void) { return 10000; }
@@ -273,77 +385,41 @@ ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t*
                         const int32_t* target_pos, int64_t T, int32_t d, int32_t V, int32_t P,
                         float* loss, float* lse, int32_t* n_valid, int32_t* dev_status,
                         void* workspace, size_t workspace_bytes, void* stream) {
-  if (!sizes_ok(T, d, V, P)) return SS_ERR_INVALID_ARG;
-  if (lm_head == nullptr || candidates == nullptr || loss == nullptr || n_valid == nullptr ||
-      dev_status == nullptr || workspace == nullptr ||
-      (T > 0 && (x == nullptr || target_pos == nullptr || lse == nullptr)))
+  return forward_impl(x, lm_head, candidates, target_pos, T, d, V, P, loss, lse, n_valid,
+                      dev_status, workspace, workspace_bytes, stream, false);
+}
+
+ss_status ss_ce_forward_e4m3(const ss_bf16* x, const ss_bf16* lm_head,
+                             const int32_t* candidates, const int32_t* target_pos, int64_t T,
+                             int32_t d, int32_t V, int32_t P, float* loss, float* lse,
+                             int32_t* n_valid, int32_t* dev_status, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  return forward_impl(x, lm_head, candidates, target_pos, T, d, V, P, loss, lse, n_valid,
+                      dev_status, workspace, workspace_bytes, stream, true);
+}
+
+size_t ss_workspace_bytes_e4m3(int64_t T, int32_t d, int32_t V, int32_t P) {
+  if (!sizes_ok(T, d, V, P) || d % 16 != 0) return 0;
+  return layout(T, d, V, P).total_e4m3;
+}
+
+ss_status ss_quantize_e4m3(const ss_bf16* src, int64_t n, uint8_t* dst, float* scale,
+                           void* scratch, void* stream) {
+  if (n < 0 || n % 8 != 0 || scale == nullptr || scratch == nullptr ||
+      (n > 0 && (src == nullptr || dst == nullptr)))
     return SS_ERR_INVALID_ARG;
-  if (!aligned16(lm_head) || !aligned16(workspace) || (T > 0 && !aligned16(x)))
-    return SS_ERR_MISALIGNED;
-  const Layout L = layout(T, d, V, P);
-  if (workspace_bytes < L.total) return SS_ERR_WORKSPACE_TOO_SMALL;
-  int sms, pairs[3];
-  ss_status ds = ensure_device(&sms, pairs);
+  if (!aligned16(src) || !aligned16(dst) || !aligned16(scratch)) return SS_ERR_MISALIGNED;
+  int sms;
+  ss_status ds = ensure_device(&sms);
   if (ds != SS_OK) return ds;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint16_t* w_c = reinterpret_cast<uint16_t*>(ws + L.w_c);
-  uint16_t* u = reinterpret_cast<uint16_t*>(ws + L.u);
-  float* ref = reinterpret_cast<float*>(ws + L.ref);
-  float* rowsum = reinterpret_cast<float*>(ws + L.rowsum);
-  float* loss_rows = reinterpret_cast<float*>(ws + L.loss_rows);
-  int32_t* fix_count = reinterpret_cast<int32_t*>(ws + L.fix_count);
-  int32_t* kstatus = dev_status + 8;
-
-  RowArgs ra{};
-  ra.rowsum = rowsum;
-  ra.ref = ref;
-  ra.tpos = target_pos;
-  ra.x = x;
-  ra.T = T;
-  ra.d = d;
-  ra.P = P;
-  ra.tiles_n = L.tiles_n;
-  ra.ldz = L.ldz;
-  ra.w_c = w_c;
-  ra.u = u;
-  ra.lse = lse;
-  ra.rscale = reinterpret_cast<float*>(ws + L.rscale);
-  ra.xs = reinterpret_cast<uint16_t*>(ws + L.xs);
-  ra.loss_rows = loss_rows;
-  ra.fix_list = reinterpret_cast<int32_t*>(ws + L.fix_list);
-  ra.fix_count = fix_count;
-  ra.partials = reinterpret_cast<double2*>(ws + L.partials);
-  ra.loss = loss;
-  ra.n_valid = n_valid;
-
-  SS_LAUNCH("gather", s, launch_gather(lm_head, candidates, P, d, V, w_c, kstatus, fix_count, 1, s));
-  if (T > 0) {
-    SS_LAUNCH("ref_logits", s, launch_ref_logits(x, w_c, target_pos, T, d, P, ref, s));
-    CUtensorMap ta, tb, tc;
-    ss_status r;
-    if ((r = make_map(&ta, x, d, T, d, 64, kBM)) != SS_OK) return r;
-    if ((r = make_map(&tb, w_c, d, P, d, 64, kBN / 2)) != SS_OK) return r;
-    if ((r = make_map(&tc, u, P, T, L.ldz, 64, 32)) != SS_OK) return r;
-    GemmArgs a{};
-    a.M = (int32_t)T;
-    a.N = P;
-    a.K = d;
-    a.tiles_m = (int32_t)((T + kBMP - 1) / kBMP);
-    a.tiles_n = L.tiles_n;
-    a.num_kb = (d + 63) / 64;
-    a.tpos = target_pos;
-    a.ref = ref;
-    a.rowsum = rowsum;
-    a.out = u;
-    a.ld_out = L.ldz;
-    a.status = kstatus;
-    const int tiles = a.tiles_m * a.tiles_n;
-    SS_LAUNCH("fwd_gemm_ce", s,
-              launch_gemm(KIND_FWD, ta, tb, tc, a, tiles < pairs[KIND_FWD] ? tiles : pairs[KIND_FWD], s));
-    SS_LAUNCH("row_pass", s, launch_rows(ra, s));
-  }
-  SS_LAUNCH("loss_finalize", s, launch_finalize(ra, s));
+  uint32_t* amax = static_cast<uint32_t*>(scratch);      // words 0..1
+  float* qs = static_cast<float*>(scratch) + 4;          // words 4..6
+  SS_CUDA(cudaMemsetAsync(amax, 0, 2 * sizeof(uint32_t), s), "cudaMemsetAsync");
+  SS_LAUNCH("amax_e4m3", s, launch_amax_bf16(src, n, nullptr, 0, amax, s));
+  SS_LAUNCH("quant_e4m3", s, launch_quant_e4m3(src, n, dst, nullptr, 0, nullptr, amax, qs, s));
+  SS_CUDA(cudaMemcpyAsync(scale, qs, sizeof(float), cudaMemcpyDeviceToDevice, s),
+          "cudaMemcpyAsync");
   return SS_OK;
 }
 
@@ -360,7 +436,7 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
     return SS_ERR_MISALIGNED;
   const Layout L = layout(T, d, V, P);
   if (workspace_bytes < L.total) return SS_ERR_WORKSPACE_TOO_SMALL;
-  int sms, pairs[3];
+  int sms, pairs[kNumGemmKinds];
   ss_status ds = ensure_device(&sms, pairs);
   if (ds != SS_OK) return ds;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

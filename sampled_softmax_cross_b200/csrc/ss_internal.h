@@ -10,6 +10,11 @@
 
 namespace ssb {
 
+// Partial row sums the forward epilogue writes per 256-column tile: one per
+// epilogue warp sharing a TMEM lane quarter (the e4m3 forward has two, each
+// over half of the tile's columns).
+constexpr int kFwdSumsPerTileBf16 = 1, kFwdSumsPerTileE4m3 = 2;
+
 // Arguments of the three tcgen05 GEMMs (forward logits, dX, dW_C).
 struct GemmArgs {
   int32_t M, N, K;           // output rows, output cols, contraction length
@@ -18,7 +23,9 @@ struct GemmArgs {
   // forward epilogue: E = exp(z - ref) and its per-tile row sums
   const int32_t* tpos;  // [M] target position of each row, -1 = ignored
   const float* ref;     // [M] reference logit of each row
-  float* rowsum;        // [tiles_n][M] sum over each 256-column tile of exp(z - ref)
+  const float* qscale;  // e4m3 forward: [2] = product of the two operand scales
+  float* rowsum;        // [tiles_n * sums per tile][M] sums of exp(z - ref) over each
+                        // tile, or over each half (128 columns) of it
   // dX / dW epilogue scale g / n (dX also times rscale[row])
   const float* grad_loss;
   const int32_t* n_valid;
@@ -34,7 +41,9 @@ struct GemmArgs {
   int32_t* status;  // dev_status + 8 (error word, detail word)
 };
 
-enum GemmKind { KIND_FWD = 0, KIND_DX = 1, KIND_DW = 2 };
+// KIND_FWD8: the forward on e4m3 operands (x and W_C quantized per tensor).
+enum GemmKind { KIND_FWD = 0, KIND_DX = 1, KIND_DW = 2, KIND_FWD8 = 3 };
+constexpr int kNumGemmKinds = 4;
 
 // Launches `pairs` CTA pairs (clusters of 2) of the persistent GEMM kernel.
 cudaError_t launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b,
@@ -61,12 +70,12 @@ cudaError_t launch_ref_logits(const uint16_t* x, const uint16_t* w_c, const int3
                               int64_t T, int32_t d, int32_t P, float* ref, cudaStream_t s);
 // Row pass after the forward GEMM (see ce_kernels.cu).
 struct RowArgs {
-  const float* rowsum;  // [tiles_n][T]
+  const float* rowsum;  // [nsums][T] partial row sums of exp(z - ref)
   const float* ref;     // [T]
   const int32_t* tpos;  // [T]
   const uint16_t* x;    // [T][d]
   int64_t T;
-  int32_t d, P, tiles_n;
+  int32_t d, P, nsums;
   int64_t ldz;
   const uint16_t* w_c;  // [P][d] (fix-up)
   uint16_t* u;          // [T][ldz] E, patched at the target column
@@ -77,6 +86,10 @@ struct RowArgs {
   int32_t* fix_list;    // [T] rows whose E overflowed
   int32_t* fix_count;   // [1]
   double2* partials;    // [kRowPartials] per-block (loss sum, valid count) of the row pass
+  // e4m3 forward (nullptr otherwise): the fix-up recomputes logits from these
+  const uint8_t* x8;    // [T][d] e4m3 codes of x
+  const uint8_t* w8;    // [P][d] e4m3 codes of W_C
+  const float* qscale;  // [3]: scale of x, of W_C, their product
   float* loss;          // [1] mean loss over valid rows
   int32_t* n_valid;     // [1]
 };
@@ -89,6 +102,17 @@ cudaError_t launch_finalize(const RowArgs& a, cudaStream_t s);
 cudaError_t launch_prefix_pos(const int32_t* prefix_table, const int32_t* targets,
                               const int32_t* vocab_pos, int64_t T, int32_t V, int32_t* prefix_pos,
                               int32_t* status, cudaStream_t s);
+// e4m3 quantization of one or two bf16 tensors (n, m multiples of 8 elements):
+// amax[0..1] must be 0 before k_amax runs; qscale[0..2] = 2^ka, 2^kb, 2^(ka+kb).
+cudaError_t launch_amax_bf16(const uint16_t* a, int64_t n, const uint16_t* b, int64_t m,
+                             uint32_t* amax, cudaStream_t s);
+cudaError_t launch_quant_e4m3(const uint16_t* a, int64_t n, uint8_t* a8, const uint16_t* b,
+                              int64_t m, uint8_t* b8, const uint32_t* amax, float* qscale,
+                              cudaStream_t s);
+// ref[i] = qscale[2] * (x8_i . w8[target_pos_i]) in fp32 (w8[0] on ignored rows).
+cudaError_t launch_ref_logits_e4m3(const uint8_t* x8, const uint8_t* w8, const int32_t* tpos,
+                                   int64_t T, int32_t d, int32_t P, const float* qscale,
+                                   float* ref, cudaStream_t s);
 cudaError_t launch_zero_rows(uint16_t* dW, int32_t V, int32_t d, const int32_t* vocab_pos,
                              int all_rows, cudaStream_t s);
 

@@ -63,11 +63,11 @@ def check_build(targets, V, P, offset, stride=20011):
     return info
 
 
-def run_path(x_bits, lm_bits, targets, P, offset, stride=20011, grad=1.0):
+def run_path(x_bits, lm_bits, targets, P, offset, stride=20011, grad=1.0, precision="bf16"):
     """build + forward + backward on the GPU; numpy results."""
     T, d = x_bits.shape
     V = lm_bits.shape[0]
-    ce = capi.SampledCE(T, d, V, P)
+    ce = capi.SampledCE(T, d, V, P, precision=precision)
     x = dev_bf16(x_bits) if T else torch.empty((1, d), dtype=torch.bfloat16, device="cuda")
     lm = dev_bf16(lm_bits)
     t = torch.from_numpy(np.ascontiguousarray(targets, dtype=np.int32)).cuda()

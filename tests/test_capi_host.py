@@ -25,7 +25,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(ss_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(ss_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_three_calls():
@@ -63,9 +63,10 @@ def test_workspace_bytes_rejects_bad_sizes(lib):
 def test_workspace_holds_logits_and_rows(lib):
     T, d, V, P = 49152, 768, 50304, 24576
     ws = capi.ss_workspace_bytes(T, d, V, P)
-    # E' [T,P] + W_C [P,d] + x' [T,d] (bf16), tile sums, per-row words, the row
+    # E' [T,P] + W_C [P,d] + x' [T,d] (bf16), two partial row sums per 256-column
+    # tile, per-row words, the row
     # pass's per-block partial sums (4096 x 16 B), builder bitmap
-    need = (T * P * 2 + P * d * 2 + T * d * 2 + ((P + 255) // 256) * T * 4 + 4 * T * 4
+    need = (T * P * 2 + P * d * 2 + T * d * 2 + 2 * ((P + 255) // 256) * T * 4 + 4 * T * 4
             + 4096 * 16)
     assert need <= ws <= need + 2 * ((V + 31) // 32) * 4 + 64 * 1024
     # padded logit rows when P is not a multiple of 8
@@ -135,3 +136,18 @@ def test_prefix_and_selftest_host_rejections(lib):
     assert f(a, None, a, 10, 100, a, a, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
     assert f(a, a, a, 10, 100, a, None, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
     assert lib.ss_selftest_wait_limit(None, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+
+
+def test_e4m3_host_rejections(lib):
+    a = ctypes.c_void_p(1 << 20)  # never dereferenced: rejected before any CUDA call
+    ws = capi.ss_workspace_bytes_e4m3(512, 128, 50304, 2048)
+    assert ws > capi.ss_workspace_bytes(512, 128, 50304, 2048) + 512 * 128 + 2048 * 128 - 1
+    assert capi.ss_workspace_bytes_e4m3(512, 136, 50304, 2048) == 0  # d % 16
+    f = lib.ss_ce_forward_e4m3
+    assert f(a, a, a, a, 512, 136, 50304, 2048, a, a, a, a, a, ws, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    assert f(a, a, a, a, 512, 128, 50304, 2048, a, a, a, a, a, ws - 1, None) == \
+        capi.STATUS["SS_ERR_WORKSPACE_TOO_SMALL"]
+    q = lib.ss_quantize_e4m3
+    assert q(a, 12, a, a, a, None) == capi.STATUS["SS_ERR_INVALID_ARG"]  # n % 8
+    assert q(a, 16, a, None, a, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
+    assert q(ctypes.c_void_p((1 << 20) + 8), 16, a, a, a, None) == capi.STATUS["SS_ERR_MISALIGNED"]
