@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsampled_ce.so")
 SOURCES = ["ss_api.cu", "ce_kernels.cu", "ce_gemm.cu", "ss_noalloc.cu"]
-HEADERS = ["sm100.cuh", "ss_internal.h"]
+HEADERS = ["sm100.cuh", "ss_internal.h", "ce_gemm.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -37,7 +37,8 @@
 //               swizzled shared-memory box and TMA stores; dX, dW: 16-byte stores)
 // Two TMEM accumulators let the epilogue of tile i overlap the MMAs of i+1.
 #include "sm100.cuh"
-#include "ss_internal.h"
+#include "ce_gemm.h"
+#include "sampled_ce.h"
 
 namespace ssb {
 
