@@ -798,27 +798,37 @@ __global__ void k_prefix_pos(const int32_t* __restrict__ prefix_table,
 // ----------------------------------------------------------------------------
 // launchers
 // ----------------------------------------------------------------------------
-static int g_sms_cache = 0;
+// Per-device launch facts (a process may drive several GPUs).
+constexpr int kMaxDevices = 128;
+static int g_sms_cache[kMaxDevices] = {};
+static bool g_build_attr[kMaxDevices] = {};
+
+static int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return (dev >= 0 && dev < kMaxDevices) ? dev : 0;
+}
+
 static int num_sms() {
-  if (g_sms_cache == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_sms_cache, cudaDevAttrMultiProcessorCount, dev);
-    if (g_sms_cache <= 0) g_sms_cache = 148;
+  const int dev = current_device();
+  if (g_sms_cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_sms_cache[dev] = n > 0 ? n : 148;
   }
-  return g_sms_cache;
+  return g_sms_cache[dev];
 }
 
 cudaError_t launch_build_mark(const int32_t* targets, int64_t T, int32_t V, int32_t P,
                               int64_t offset, int32_t stride, uint32_t* bitmap, int32_t* prefix,
                               int32_t* dev_status, cudaStream_t s) {
   const int smem = ((V + 31) / 32) * 4;
-  static bool attr = false;
-  if (!attr) {
+  const int dev = current_device();
+  if (!g_build_attr[dev]) {  // the attribute is per device
     cudaError_t e = cudaFuncSetAttribute(k_build_mark, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (SS_MAX_VOCAB / 32) * 4);
     if (e != cudaSuccess) return e;
-    attr = true;
+    g_build_attr[dev] = true;
   }
   k_build_mark<<<1, kBuildThreads, smem, s>>>(targets, T, V, P, offset, stride, bitmap, prefix,
                                               dev_status);
