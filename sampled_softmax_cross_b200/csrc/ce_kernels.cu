@@ -499,15 +499,15 @@ __global__ void k_ref_logits_e4m3(const uint4* __restrict__ x8, const uint4* __r
 }
 
 // ----------------------------------------------------------------------------
-// Row pass after the forward GEMM. With S_i = sum of the row's per-tile sums of
-// exp(z - ref_i):
+// Row pass after the forward GEMM. With S_i = sum of the row's partial sums of
+// exp(z - ref_i) (one per tile, or per half tile in the e4m3 forward):
 //   lse_i = ref_i + log S_i,   loss_i = lse_i - z_target = log S_i (valid rows),
 //   r_i = 1 / S_i (0 on ignored rows),  E'[i, t_i] = 1 - S_i,  x'_i = r_i x_i,
 // so that r_i E'_ij = softmax_ij - [j == t_i] (the CE gradient w.r.t. the
 // logits, "Learning Triton One Kernel at a Time: Softmax", section "Gradient")
 // and the backward is dX = (g/n) r (.) (E' W_C), dW_C = (g/n) E'^T x'.
 // A row whose S_i is not below 2^64 (E overflowed: its loss exceeds ~44 nats)
-// is listed for the exact fix-up below instead.
+// is listed for the exact fix-up in k_finalize instead.
 // ----------------------------------------------------------------------------
 constexpr float kFixThreshold = 1.8446744e19f;  // 2^64
 
@@ -520,9 +520,9 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 a, float r) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Each warp takes 8 consecutive rows. For the tile sums (stored tile-major)
-// lane l adds tiles (l / 8), (l / 8) + 4, ... of row (l % 8), so every load
-// instruction reads whole 32-byte sectors; the four partial sums of a row are
+// Each warp takes 8 consecutive rows. For the partial sums (stored sum-major)
+// lane l adds sums (l / 8), (l / 8) + 4, ... of row (l % 8), so every load
+// instruction reads whole 32-byte sectors; the four lane totals of a row are
 // then combined in a fixed order. The x' rows are written 4 at a time with
 // all their loads in flight.
 constexpr int kRowsPerWarp = 8;
