@@ -527,7 +527,7 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 a, float r) {
 // all their loads in flight.
 constexpr int kRowsPerWarp = 8;
 
-__global__ void __launch_bounds__(256) k_rows(RowArgs a) {
+__global__ void __launch_bounds__(256, 3) k_rows(RowArgs a) {
   __shared__ double2 s_part[8];
   const int lane = threadIdx.x & 31;
   const int vpr = a.d / 8;
@@ -540,8 +540,18 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a) {
     const int64_t r = gidx * kRowsPerWarp + (lane & 7);
     const bool in = r < a.T;
     float s = 0.f;
-    if (in)
-      for (int t = lane >> 3; t < a.nsums; t += 4) s += __ldg(a.rowsum + (int64_t)t * a.T + r);
+    if (in) {
+      // eight loads in flight per batch, added in the order of t
+      int t = lane >> 3;
+      for (; t + 28 < a.nsums; t += 32) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldg(a.rowsum + (int64_t)(t + 4 * u) * a.T + r);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s += v[u];
+      }
+      for (; t < a.nsums; t += 4) s += __ldg(a.rowsum + (int64_t)t * a.T + r);
+    }
     s += __shfl_xor_sync(0xffffffffu, s, 8);
     s += __shfl_xor_sync(0xffffffffu, s, 16);
     const float S = s;  // identical in the four lanes of the row
