@@ -3,12 +3,12 @@
  * cross-entropy LM head: candidate build, forward and backward.
  *
  * The method is the one of "sampled_softmax.py" (modded-nanogpt,
- * track_1_short): every token of a microbatch shares one candidate set C of
- * P classes -- every class that is a target somewhere in the microbatch, plus
- * negatives taken from the next window of the stride permutation
- * k * stride mod V -- and the cross-entropy is a softmax over C instead of
- * the whole vocabulary (module docstring, "What"). The lm_head gradient is
- * dense over the vocabulary with zeros outside C.
+ * track_1_short): all tokens of a microbatch use one candidate set C of P
+ * classes -- the classes that occur as targets in the microbatch, topped up
+ * with negatives read from the stride permutation k * stride mod V, a window
+ * that moves on every build -- and the cross-entropy normalises over C rather than the
+ * whole vocabulary (module docstring, "What"). The lm_head gradient covers
+ * all V rows, with exact zeros in the rows of classes not in C.
  *
  * Conventions for every entry point
  *   - All array arguments are DEVICE pointers on the current CUDA device,
@@ -79,8 +79,9 @@ typedef enum ss_status {
  * are invalid). One workspace serves ss_build_candidates, ss_ce_forward and
  * ss_ce_backward of the same microbatch; ss_ce_forward leaves the gathered
  * rows W_C and the gradient factors (below) in it for ss_ce_backward, so it must not be
- * reused between a forward and its backward (the "one microbatch per step"
- * contract of sampled_softmax.py, SampledSoftmax.__init__). */
+ * reused between a forward and its backward (sampled_softmax.py,
+ * SampledSoftmax.__init__, keeps the same rule: a single microbatch in flight
+ * per step). */
 SS_API size_t ss_workspace_bytes(int64_t T, int32_t d, int32_t V, int32_t P);
 
 /* Bytes of workspace ss_build_candidates alone needs for a vocabulary of V
@@ -93,8 +94,8 @@ SS_API size_t ss_build_workspace_bytes(int32_t V);
  *   if D < P take need = P - D negatives: the first `need` unmarked classes of
  *   the stride sweep c_k = (stride * k) mod V for k = offset, offset+1, ...,
  *   offset+draw-1 (k mod V), draw = min(V, floor(1.7 * need) + 256); if that
- *   window holds fewer than `need` unmarked classes, take instead
- *   free[0 :: max(1, |free| / need)][:need] over the ascending unmarked classes.
+ *   window holds fewer than `need` unmarked classes, take instead every s-th
+ *   ascending unmarked class from the first, s = max(1, #unmarked / need).
  *   C = marked classes in ascending order.
  * In:  targets [T] int32, each in [-1, V) (-1 = ignored token);
  *      offset >= 0 (reduced mod V); stride coprime with V (SS_DEFAULT_STRIDE).
@@ -194,7 +195,7 @@ SS_API ss_status ss_quantize_e4m3(const ss_bf16* src, int64_t n, uint8_t* dst, f
  *   G     = (g / n_valid) * (softmax - onehot)  (0 when n_valid = 0);
  *   dx    = G @ W_C                      [T, d] bf16;
  *   dW    = dense [V, d] bf16: row C_j = (G^T @ x)_j, every other row +0.0
- *           (module docstring: "dense over the vocabulary with zeros outside C").
+ *           (module docstring: the lm_head gradient spans the vocabulary).
  * Computed from the forward's workspace as dx = (g/n) r (.) (E' @ W_C) and
  * dW_C = (g/n) E'^T @ x'.
  * In:  grad_loss [1] float32 (device); candidates, vocab_pos as above; n_valid
@@ -216,12 +217,12 @@ SS_API const char* ss_last_cuda_error(void);
 /* Library version, major * 10000 + minor * 100 + patch. */
 SS_API int32_t ss_version(void);
 
-/* Positions in C of each token's prefix target (sampled_softmax.py: module
+/* Where each token's prefix target sits in C (sampled_softmax.py: module
  * docstring, CandidateBuilder.build and the SampledLoss field prefix_pos).
  * For token i with a valid target t_i the prefix target is
  * p_i = prefix_table[t_i]; prefix_pos[i] = vocab_pos[p_i] when p_i is a class
- * of C, and -1 otherwise: when p_i is a class outside C (the prefix target is
- * dropped for that token, so prefix targets never add classes to C), when
+ * of C, and -1 otherwise: when p_i is a class outside C (that token then has
+ * no prefix target, and prefix targets never add classes to C), when
  * p_i = -1 ("no prefix"), and for an ignored token (t_i = -1). The caller's
  * loss reads -1 as a no-op.
  * In:  prefix_table [V] int32, entries in [-1, V); targets [T] and vocab_pos

@@ -35,7 +35,7 @@ import numpy as np
 
 NEGATIVE_STRIDE = 20011
 
-# Window length factor and pad: ``draw = min(V, int(need * 1.7) + 256)``
+# Window length factor and pad: draw = min(V, floor(1.7 need) + 256) positions
 # (sampled_softmax.py, CandidateBuilder._negatives).
 WINDOW_FACTOR = 1.7
 WINDOW_PAD = 256
@@ -75,9 +75,9 @@ def pick_negatives(mark: np.ndarray, need: int, offset: int, V: int, stride: int
     The window is the next ``draw`` positions of the stride sweep starting at
     ``offset``. Classes already marked (the targets) are skipped; the first
     ``need`` survivors, in sweep order, are the negatives. When the window
-    holds fewer than ``need`` survivors, the fallback takes an evenly strided
-    pick over all unmarked classes in ascending order:
-    ``free[::max(1, len(free) // need)][:need]``.
+    holds fewer than ``need`` survivors, the fallback walks all unmarked
+    classes in ascending order and keeps every s-th one, starting with the
+    first, s = max(1, floor(#unmarked / need)), until it has ``need``.
 
     Returns (negatives, draw, used_fallback). ``mark`` is not modified: the
     window is tested against the targets' marks only, as on the page.
@@ -89,7 +89,7 @@ def pick_negatives(mark: np.ndarray, need: int, offset: int, V: int, stride: int
         return survivors[:need], draw, False
     free = np.flatnonzero(~mark)
     if free.size < need:
-        raise OracleError("no_free_classes", f"only {free.size} free classes for {need}")
+        raise OracleError("no_free_classes", f"{need} negatives wanted, {free.size} unmarked classes left")
     step = max(1, free.size // need)
     return free[::step][:need], draw, True
 
@@ -99,7 +99,7 @@ def build_candidates(targets: np.ndarray, V: int, P: int, offset: int = 0,
     """Candidate set C and its maps for one microbatch (CandidateBuilder.build).
 
     Steps, in the page's order:
-      1. mark every class that is a target (``-1`` = no target, skipped);
+      1. mark the classes that occur as targets (``-1`` = none, skipped);
       2. num_targets D = number of marked classes; D > P is an error;
       3. if D != P, mark P - D negatives from the stride window (pick_negatives);
       4. C = the marked classes in ascending order;
@@ -148,9 +148,9 @@ def build_candidates(targets: np.ndarray, V: int, P: int, offset: int = 0,
 
 def prefix_positions(prefix_table: np.ndarray, targets: np.ndarray,
                      vocab_pos: np.ndarray) -> np.ndarray:
-    """Position in C of each token's prefix target (CandidateBuilder.build, and
-    the SampledLoss field ``prefix_pos``; module docstring: a prefix target not
-    in C is dropped for that token, so it never forces a class into C).
+    """Where each token's prefix target sits in C (CandidateBuilder.build, and
+    the SampledLoss field ``prefix_pos``; module docstring: a token whose
+    prefix class is not in C gets no prefix target; it never adds a class).
 
     Steps, in the page's order:
       1. prefix target of token i = prefix_table[targets[i]];
@@ -253,8 +253,8 @@ def sampled_ce_backward(grad_loss: float, x: np.ndarray, w_c: np.ndarray,
                         logit_x: np.ndarray | None = None, logit_w: np.ndarray | None = None):
     """dX = G @ W_C and the dense lm_head gradient dW (zeros outside C).
 
-    Module docstring of sampled_softmax.py: "two gradient GEMMs" and "the
-    gradient for lm_head is dense over the vocabulary with zeros outside C".
+    Module docstring of sampled_softmax.py: the two gradient GEMMs, and an
+    lm_head gradient over every vocabulary row that is zero off C.
     dW_C = G^T @ x is accumulated over row chunks; dW[C_j] = dW_C[j].
     G comes from the logits z = logit_x @ logit_w^T, by default x and W_C
     themselves (the e4m3 variant passes its quantized operands here).

@@ -6,8 +6,8 @@
 //   dX      : dx[T,d]   = r (.) (E'[T,P] . W_C)   epilogue: per-row scale
 //   dW      : dW_C[P,d] = E'^T . x'[T,d]          epilogue: row scatter into dW[V,d]
 //
-// sampled_softmax.py (module docstring, "What"/"Why") names these as the
-// logits GEMM, the CE pass and the "two gradient GEMMs".
+// sampled_softmax.py (module docstring, "What"/"Why") counts them as the
+// logits GEMM with its CE pass, and the pair of gradient GEMMs.
 //
 // The forward never stores the logits. Each row i has a reference logit ref_i
 // computed beforehand (the logit of its target class), and the epilogue
