@@ -29,12 +29,15 @@
 // CTAs on one TPC, tcgen05 cta_group::2). Each CTA loads its own 128 rows of A
 // and its 128-column half of B; the pair's leader issues M=256, N=256, K=16
 // MMAs that read both CTAs' shared memory and write 128 rows x 256 fp32
-// columns into each CTA's TMEM. Per CTA, 192 threads, persistent over tiles:
-//   warp 0      TMA producer, ring of 32 KB stages (A 128x64 + B 128x64):
-//               6 in the forward, 7 in dX and dW
+// columns into each CTA's TMEM. Per CTA, persistent over tiles:
+//   warp 0      TMA producer, ring of 32 KB stages (A 128x64 + B 128x64 bf16,
+//               or 128x128 e4m3 codes): 6 in the forward, 5 in the e4m3
+//               forward, 7 in dX and dW
 //   warp 1      TMEM owner (2 x 256 columns); in the leader, the MMA issuer
-//   warps 2..5  epilogue: TMEM -> registers -> math -> global (forward: through a
-//               swizzled shared-memory box and TMA stores; dX, dW: 16-byte stores)
+//               (kind::f16, or kind::f8f6f4 with K=32 for the e4m3 forward)
+//   warps 2..   epilogue, 4 warps (8 in the e4m3 forward, two per TMEM lane
+//               quarter): TMEM -> registers -> math -> global (forward: through
+//               swizzled shared-memory boxes and TMA stores; dX, dW: 16-byte stores)
 // Two TMEM accumulators let the epilogue of tile i overlap the MMAs of i+1.
 #include "sm100.cuh"
 #include "ce_gemm.h"

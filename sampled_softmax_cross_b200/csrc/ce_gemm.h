@@ -17,7 +17,7 @@ constexpr int kFwdSumsPerTileBf16 = 1, kFwdSumsPerTileE4m3 = 2;
 struct GemmArgs {
   int32_t M, N, K;           // output rows, output cols, contraction length
   int32_t tiles_m, tiles_n;  // ceil(M / 256) (CTA-pair rows), ceil(N / 256)
-  int32_t num_kb;            // ceil(K / 64)
+  int32_t num_kb;            // K blocks: ceil(K / 64), ceil(K / 128) for e4m3
   // forward epilogue: E = exp(z - ref) and its per-tile row sums
   const int32_t* tpos;  // [M] target position of each row, -1 = ignored
   const float* ref;     // [M] reference logit of each row
@@ -28,8 +28,8 @@ struct GemmArgs {
   const float* grad_loss;
   const int32_t* n_valid;
   const float* rscale;  // [M] (dX) 1 / S_i, 0 on ignored rows
-  // forward / dX epilogue without TMA store: output rows
-  uint16_t* out;        // [M][ld_out] bf16 (E for the forward, dx for dX)
+  // epilogues that store from registers (dX): output rows
+  uint16_t* out;        // [M][ld_out] bf16 (dx; the forward's E when stored so)
   int64_t ld_out;
   // dW epilogue
   const int32_t* cand;       // [M] class id of each output row
