@@ -143,3 +143,16 @@ def test_e4m3_headline_workload():
     dw_o = oc.dw_c_rows(x, w_c, tpos, lse, scale, cols, logit_x=xq, logit_w=wq)
     dw_g = wl.bits_to_f64(g["dW_bits"][cand[cols]])
     assert rel_fro(dw_g, dw_o) <= GRAD_RTOL, rel_fro(dw_g, dw_o)
+
+
+def test_e4m3_empty_microbatch_and_full_vocabulary():
+    lm = wl.bf16_bits(np.random.default_rng(0).standard_normal((512, 64), dtype=np.float32))
+    g = run_path(np.zeros((0, 64), np.uint16), lm, np.zeros(0, np.int32), 100, 4,
+                 precision="e4m3")
+    assert g["loss"] == 0.0 and g["n_valid"] == 0 and np.all(g["dW_bits"] == 0)
+    # P = V: C is the whole vocabulary, the e4m3 loss is the full CE on e4m3 logits
+    x, lm, t = wl.make_inputs(300, 64, 777, 1.1, 0.05, 8)
+    g = run_path(x, lm, t, 777, 0, precision="e4m3")
+    o = _e4m3_oracle(x, lm, t, 777, 0)
+    assert np.array_equal(o["candidates"], np.arange(777))
+    compare_full(g, o, t)
