@@ -489,6 +489,13 @@ def run_ours(args, w):
             "gpu_launches": launches,
             "clocks": clk,
             "clock_normalized": clock_normalized(step_tflops, per, clk, world),
+            "context": {
+                "pages_claim": "with P = 10k-25k candidates the logits GEMM, the CE pass and the "
+                               "two gradient GEMMs shrink 2-5x against the full softmax over "
+                               "V = 50304 (no hardware stated)",
+                "V_over_P": w.V / w.P,
+                "measured": "profiles/candidate_count_vs_full_softmax.md",
+            },
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
