@@ -62,9 +62,19 @@ __device__ __forceinline__ void write_status(int32_t* st, int code, int D, int n
   for (int i = 8; i < SS_DEV_STATUS_WORDS; ++i) st[i] = 0;
 }
 
-// One CTA: target bitmap in shared memory, D, negative window or fallback,
-// then the bitmap and its per-word exclusive popcount prefix go to global.
-__global__ void __launch_bounds__(kBuildThreads)
+__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
+// A cluster of kBuildCluster CTAs marks the targets, each its share into its
+// own shared-memory bitmap; CTA 0 then ORs the others' bitmaps in (distributed
+// shared memory) and alone goes on: D, negative window or fallback, and the
+// bitmap with its per-word exclusive popcount prefix to global.
+constexpr int kBuildCluster = 8;
+
+__global__ void __cluster_dims__(kBuildCluster, 1, 1) __launch_bounds__(kBuildThreads)
     k_build_mark(const int32_t* __restrict__ targets, int64_t T, int32_t V, int32_t P,
                  int64_t offset, int32_t stride, uint32_t* __restrict__ g_bitmap,
                  int32_t* __restrict__ g_prefix, int32_t* __restrict__ st) {
@@ -73,22 +83,25 @@ __global__ void __launch_bounds__(kBuildThreads)
   __shared__ int s_bad;
   const int tid = threadIdx.x;
   const int NW = (V + 31) >> 5;
+  const uint32_t crank = cluster_ctarank();
 
   for (int w = tid; w < NW; w += kBuildThreads) bm[w] = 0u;
   if (tid == 0) s_bad = INT_MAX;
   __syncthreads();
 
-  // 1. mark every valid target (-1 = ignored; anything else outside [0, V) is an error)
+  // 1. mark this CTA's share of the valid targets (-1 = ignored; anything
+  //    else outside [0, V) is an error)
   {
     const int64_t n4 = T >> 2;
+    const int64_t v_lo = n4 * crank / kBuildCluster, v_hi = n4 * (crank + 1) / kBuildCluster;
     const int4* t4 = reinterpret_cast<const int4*>(targets);
     // 8 vector loads in flight per thread before the shared-memory atomics
-    for (int64_t i0 = tid; i0 < n4; i0 += 8 * kBuildThreads) {
+    for (int64_t i0 = v_lo + tid; i0 < v_hi; i0 += 8 * kBuildThreads) {
       int4 q[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int64_t i = i0 + (int64_t)u * kBuildThreads;
-        q[u] = i < n4 ? __ldg(t4 + i) : make_int4(-1, -1, -1, -1);
+        q[u] = i < v_hi ? __ldg(t4 + i) : make_int4(-1, -1, -1, -1);
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -107,7 +120,7 @@ __global__ void __launch_bounds__(kBuildThreads)
         }
       }
     }
-    for (int64_t i = 4 * n4 + tid; i < T; i += kBuildThreads) {
+    for (int64_t i = 4 * n4 + tid; crank == 0 && i < T; i += kBuildThreads) {
       const int t = __ldg(targets + i);
       if (t == -1) continue;
       if (t < -1 || t >= V) {
@@ -118,6 +131,20 @@ __global__ void __launch_bounds__(kBuildThreads)
     }
   }
   __syncthreads();
+  cluster_sync();  // every CTA's marks are in its shared memory
+  if (crank == 0) {
+    for (int w = tid; w < NW; w += kBuildThreads) {
+      uint32_t v = bm[w];
+      const uint32_t a = smem_u32(&bm[w]);
+#pragma unroll
+      for (int r = 1; r < kBuildCluster; ++r) v |= ld_dsmem_u32(mapa_shared(a, r));
+      bm[w] = v;
+    }
+    if (tid > 0 && tid < kBuildCluster)
+      atomicMin(&s_bad, (int)ld_dsmem_u32(mapa_shared(smem_u32(&s_bad), tid)));
+  }
+  cluster_sync();  // CTA 0 has read the others' shared memory
+  if (crank != 0) return;
   if (s_bad != INT_MAX) {
     if (tid == 0) write_status(st, SS_ERR_BAD_TARGET, 0, 0, 0, 0, (int)offset, s_bad, 0);
     return;
@@ -840,8 +867,8 @@ cudaError_t launch_build_mark(const int32_t* targets, int64_t T, int32_t V, int3
     if (e != cudaSuccess) return e;
     g_build_attr[dev] = true;
   }
-  k_build_mark<<<1, kBuildThreads, smem, s>>>(targets, T, V, P, offset, stride, bitmap, prefix,
-                                              dev_status);
+  k_build_mark<<<kBuildCluster, kBuildThreads, smem, s>>>(targets, T, V, P, offset, stride,
+                                                          bitmap, prefix, dev_status);
   return cudaGetLastError();
 }
 
