@@ -253,9 +253,11 @@ SS_API ss_status ss_selftest_wait_limit(int32_t* dev_status, void* stream);
 
 /* Kernel timing for diagnostics. While enabled, each kernel launch the library
  * makes is bracketed by two CUDA events recorded on its stream (a pool of
- * 8192 launches; later launches go untimed). ss_timing_query synchronises on
- * the recorded events and returns, for the i-th distinct kernel name, its
- * launch count and total milliseconds. Not thread-safe; for benchmarks. */
+ * 8192 launches; later launches go untimed); enable = 2 brackets only the
+ * tensor-core GEMM launches (fewer events in a timed loop), 1 every launch,
+ * 0 none. ss_timing_query synchronises on the recorded events and returns,
+ * for the i-th distinct kernel name, its launch count and total
+ * milliseconds. Not thread-safe; for benchmarks. */
 SS_API ss_status ss_timing_enable(int32_t enable);
 SS_API ss_status ss_timing_reset(void);
 SS_API int32_t ss_timing_count(void);

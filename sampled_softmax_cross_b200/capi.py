@@ -209,8 +209,10 @@ def ss_version() -> int:
     return int(load().ss_version())
 
 
-def ss_timing_enable(on: bool):
-    _check("ss_timing_enable", load().ss_timing_enable(1 if on else 0))
+def ss_timing_enable(on, gemms_only: bool = False):
+    """Bracket each launch with CUDA events (only the GEMM launches if gemms_only)."""
+    mode = (2 if gemms_only else 1) if on else 0
+    _check("ss_timing_enable", load().ss_timing_enable(mode))
 
 
 def ss_timing_reset():

@@ -111,6 +111,7 @@ ss_status make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
 // ----------------------------------------------------------------- timing --
 struct TimingState {
   bool on = false;
+  bool gemms_only = false;  // enable == 2: time only the tensor-core GEMM launches
   std::vector<cudaEvent_t> ev;        // pairs
   std::vector<int> rec_name;          // name index per used pair
   std::vector<std::string> names;
@@ -121,6 +122,7 @@ constexpr size_t kTimingPairs = 8192;
 
 int timing_begin(const char* name, cudaStream_t s) {
   if (!g_tm.on || g_tm.used >= kTimingPairs) return -1;
+  if (g_tm.gemms_only && strstr(name, "gemm") == nullptr) return -1;
   if (g_tm.ev.empty()) {
     g_tm.ev.resize(2 * kTimingPairs);
     for (auto& e : g_tm.ev) cudaEventCreate(&e);
@@ -523,6 +525,7 @@ ss_status ss_selftest_wait_limit(int32_t* dev_status, void* stream) {
 
 ss_status ss_timing_enable(int32_t enable) {
   g_tm.on = enable != 0;
+  g_tm.gemms_only = enable == 2;
   return SS_OK;
 }
 

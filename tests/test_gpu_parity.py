@@ -282,6 +282,14 @@ def test_kernel_timing_records_every_kernel():
     for k in names:
         assert rec[k][0] == 1 and rec[k][1] > 0, (k, rec)
     assert set(rec) == set(names), rec  # the dW GEMM writes the zero rows itself
+    capi.ss_timing_enable(True, gemms_only=True)
+    try:
+        run_path(x, lm, t, 1024, 0)
+    finally:
+        capi.ss_timing_enable(False)
+    rec = capi.ss_timing_read()
+    capi.ss_timing_reset()
+    assert set(rec) == {"fwd_gemm_ce", "dx_gemm", "dw_gemm_scatter"}, rec
 
 
 # ------------------------------------------------ full-size workloads --
