@@ -9,8 +9,11 @@ dense-contraction work of a step is 6*T*d*P FLOPs.
     python bench.py --impl reference ...   # the float64 CPU oracle, bounded sample
 
 With N > 1 (launched by torch.distributed.run) every rank runs its own
-microbatch (seed + rank, negative-window offset staggered by V*rank/N); the
-path has no collective, so this is weak scaling, timed as the max over ranks.
+microbatch (seed + rank, negative-window offset staggered by V*rank/N): weak
+scaling, timed as the max over ranks. The path itself has no collective; the
+data-parallel gradient sync of the dense dW [V, d] (an NCCL all-reduce, on its
+own stream, overlapping the next step's build and forward) runs inside the
+timed region unless --no-dp-allreduce is given.
 """
 
 from __future__ import annotations
@@ -48,6 +51,8 @@ def parse():
     ap.add_argument("--precision", choices=["bf16", "e4m3"], default="bf16",
                     help="operands of the logits GEMM (e4m3: per-tensor scaled 8-bit floats; "
                          "the gradient GEMMs stay bf16)")
+    ap.add_argument("--no-dp-allreduce", action="store_true",
+                    help="with N > 1: leave out the NCCL all-reduce of dW after each step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256,
@@ -87,6 +92,77 @@ def clock_normalized(step_tflops, per, clk, world):
         if k in per and "tflops" in per[k]:
             out[k + "_frac"] = per[k]["tflops"] / (f8 * peak / world)
     return out
+
+class NvmlClockSampler:
+    """SM clock, power and clock-event reasons read in-process through NVML
+    every `period` seconds while the timed region runs. It only reads: no
+    clock, power limit or other setting of the GPU is changed."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4),
+               ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, dev, period: float = 0.01):
+        import pynvml
+        import torch
+
+        self.nv = pynvml
+        self.period = period
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(dev)
+        try:
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(dev.index or 0)
+        self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.rows = []
+
+    def _sample(self):
+        nv = self.nv
+        return (float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)),
+                int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)),
+                nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0)
+
+    def start(self):
+        import threading
+        self.rows = [self._sample()]
+        self.stop_flag = threading.Event()
+
+        def loop():
+            while not self.stop_flag.wait(self.period):
+                try:
+                    self.rows.append(self._sample())
+                except Exception:
+                    break
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        try:
+            self.rows.append(self._sample())
+        except Exception:
+            pass
+        rows = self.rows
+        counts = {name: sum(1 for _, r, _ in rows if r & bit) for name, bit in self.REASONS}
+        return {"sm_mhz": float(np.median([c for c, _, _ in rows])),
+                "sm_min_mhz": min(c for c, _, _ in rows), "sm_max_mhz": self.sm_max,
+                "reasons": sorted(k for k, v in counts.items() if v),
+                "reason_samples": {k: v for k, v in counts.items() if v},
+                "power_w_median": float(np.median([p for _, _, p in rows])),
+                "samples": len(rows), "period_ms": self.period * 1e3, "source": "nvml"}
+
+
+def clock_sampler(dev):
+    """The in-process NVML sampler, else nvidia-smi at 100 ms."""
+    try:
+        return NvmlClockSampler(dev)
+    except Exception:
+        return ClockSampler(dev.index if dev.index is not None else 0)
+
 
 class ClockSampler:
     """nvidia-smi clock and throttle-reason samples taken while the timed region runs."""
@@ -211,7 +287,7 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, args.gpus),
+        "config": workload_config(w, args.gpus, args.gpus > 1 and not args.no_dp_allreduce),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -220,11 +296,13 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w, n):
+def workload_config(w, n, dp=False):
     return {"workload": f"{w.name}: T={w.T} d={w.d} V={w.V} P={w.P} (per rank)",
             "T": w.T, "d": w.d, "V": w.V, "P": w.P, "offset": w.offset, "zipf_s": w.zipf_s,
             "ignored_frac": w.ignore_frac, "seed": w.seed,
-            "parallelism": f"dp{n} (independent microbatch per rank, no collective)",
+            "parallelism": (f"dp{n} (independent microbatch per rank" +
+                            (", dW all-reduced over the ranks after each step)" if n > 1 and dp
+                             else ", no collective)")),
             "l2": "no explicit flush: each step streams >2 GB of bf16 logits through HBM (L2 126 MB)"}
 
 
@@ -253,7 +331,7 @@ def traffic_for(kernel):
     return rec.get("bytes_per_launch_full_size"), rec.get("note")
 
 
-def run_e2e(args, w, world, dev, x_bits, lm_bits, targets, offset, barrier, dist, ce0):
+def run_e2e(args, w, world, dev, x_bits, lm_bits, targets, offset, barrier, dist, ce0, dp=False):
     """The same step from pinned host buffers, as a training loop runs it.
 
     Every step copies its inputs (x, lm_head, targets) host -> device and its
@@ -293,6 +371,8 @@ def run_e2e(args, w, world, dev, x_bits, lm_bits, targets, offset, barrier, dist
         comp.wait_event(b["h2d"])
         comp.wait_event(b["d2h"])  # step k-2's results have left these buffers
         b["ce"].step(b["t"], b["x"], b["lm"], offset, stream=comp)
+        if dp:  # the data-parallel gradient sync, on the compute stream here
+            ranks.allreduce_dw(b["ce"].dW, dist)
         b["done"].record(comp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(b["done"])
@@ -345,6 +425,7 @@ def run_ours(args, w):
     if world > 1:
         dist.barrier()
     capi.load()
+    dp = world > 1 and not args.no_dp_allreduce
 
     # this rank's microbatch: own seed, staggered window start
     x_bits, lm_bits, targets = wl.make_inputs(w.T, w.d, w.V, w.zipf_s, w.ignore_frac,
@@ -356,37 +437,74 @@ def run_ours(args, w):
     ce = capi.SampledCE(w.T, w.d, w.V, w.P, device=dev, precision=args.precision)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        ce.step(t, x, lm, offset, stream=stream)
+    # Data-parallel gradient sync (N > 1): step k's dW (one of two buffers) is
+    # summed over the ranks on a communication stream while step k+1 builds
+    # and runs its forward; step k+2's backward waits for that sum before it
+    # rewrites the buffer.
+    dws = [ce.dW, torch.empty_like(ce.dW)] if dp else [ce.dW]
+    comm = torch.cuda.Stream(dev) if dp else None
+    ar_done = [torch.cuda.Event() for _ in dws]
+    ar_ev = []  # (start, end) events of the all-reduces in the timed loop
+
+    def step(k, timed_ar=False):
+        buf = k % len(dws)
+        ce.build(t, offset, stream=stream)
+        ce.forward(x, lm, stream=stream)
+        if dp:
+            stream.wait_event(ar_done[buf])
+        ce.backward(stream=stream, dW=dws[buf])
+        if dp:
+            comm.wait_stream(stream)
+            if timed_ar:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(comm)
+            ranks.allreduce_dw(dws[buf], dist, stream=comm)
+            if timed_ar:
+                e1.record(comm)
+                ar_ev.append((e0, e1))
+            ar_done[buf].record(comm)
+
+    def drain():
+        if dp:
+            for e in ar_done:
+                stream.wait_event(e)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        step()
+    for k in range(args.warmup):
+        step(k)
+    drain()
     torch.cuda.synchronize(dev)
     st = ce.status()
     if st[0] != 0 or st[8] != 0:
         raise RuntimeError(f"device status {st}")
 
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    # Inside the timed loop only the GEMM launches carry timing events (the
-    # roofline kernel is one of them); the small kernels are timed in a short
-    # separate pass below, so the loop pays for 6 events per step, not 18.
+    clocks = clock_sampler(dev)
+    # Inside the timed loop only the three GEMM launches carry timing events
+    # (the roofline kernel is one of them), plus one event per step boundary
+    # for the per-step times; the small kernels are timed in a short separate
+    # pass below. The library creates its events when timing is switched on,
+    # before the loop.
     capi.ss_timing_reset()
     capi.ss_timing_enable(True, gemms_only=True)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     clocks.start()
     barrier()
     torch.cuda.synchronize(dev)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
+    evs[0].record(stream)
+    for k in range(args.steps):
+        step(k, timed_ar=True)
+        evs[k + 1].record(stream)
+    drain()
+    ev_end = torch.cuda.Event(enable_timing=True)
+    ev_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    ms = ev0.elapsed_time(ev1)
+    ms = evs[0].elapsed_time(ev_end)
+    step_ms = [evs[k].elapsed_time(evs[k + 1]) for k in range(args.steps)]
+    ar_ms = [a.elapsed_time(b) for a, b in ar_ev]
     clk = clocks.stop()
     capi.ss_timing_enable(False)
     kernels = capi.ss_timing_read()
@@ -394,12 +512,14 @@ def run_ours(args, w):
     # every kernel, timed over a short pass after the timed loop
     n_sep = max(10, args.steps // 10)
     capi.ss_timing_enable(True)
-    for _ in range(n_sep):
-        step()
+    for k in range(n_sep):
+        step(k)
+    drain()
     torch.cuda.synchronize(dev)
     capi.ss_timing_enable(False)
     every = capi.ss_timing_read()
     capi.ss_timing_reset()
+    timed_in_loop = set(kernels)
     for k, (n, tot) in every.items():
         if k not in kernels:  # small kernels: per-launch time from the separate pass
             kernels[k] = (n * args.steps // n_sep, tot / n * (n * args.steps // n_sep))
@@ -407,16 +527,24 @@ def run_ours(args, w):
     launches = sum(n for n, _ in every.values()) * args.steps // n_sep
 
     ms_max = ranks.max_over_ranks(ms, dist if world > 1 else None, dev)
+    med_max = ranks.max_over_ranks(float(np.median(step_ms)), dist if world > 1 else None, dev)
 
     # e2e: the same step from pinned host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, w, world, dev, x_bits, lm_bits, targets, offset, barrier, dist, ce)
+        e2e = run_e2e(args, w, world, dev, x_bits, lm_bits, targets, offset, barrier, dist, ce,
+                      dp)
 
     if rank == 0:
         pk = peaks()
         tokens = w.T * world * args.steps
         value = tokens / (ms_max / 1e3)
+        # A kernel timed in a region shorter than a second runs at the burst
+        # clock; the sustained (seconds-long, power-capped) peak applies to
+        # longer regions.
+        burst = ms_max < 1000.0
+        tpk = pk["bf16"] if burst else pk["bf16_sus"]
+        tpk_name = "burst" if burst else "sustained"
         per = {}
         flops_gemm = 2.0 * w.T * w.d * w.P
         alg = {  # algorithmic work per launch
@@ -437,15 +565,16 @@ def run_ours(args, w):
         total_k = sum(t for _, t in kernels.values())
         for k, (n, tot) in kernels.items():
             avg = tot / max(n, 1)
-            e = {"launches": n, "avg_ms": avg, "share": tot / total_k if total_k else None}
+            e = {"launches": n, "avg_ms": avg, "share": tot / total_k if total_k else None,
+                 "timed": "in the timed loop" if k in timed_in_loop
+                 else f"separate pass of {n_sep} steps (scaled to {args.steps})"}
             if k in alg:
                 bound, work = alg[k]
-                if bound == "tensor":
+                if bound in ("tensor", "tensor8"):
+                    f8 = 2.0 if bound == "tensor8" else 1.0
                     e["tflops"] = work / (avg / 1e3) / 1e12
-                    e["frac_of_sustained"] = e["tflops"] / pk["bf16_sus"]
-                elif bound == "tensor8":  # e4m3: twice the bf16 rate (2.25 -> 4.5 PF nominal)
-                    e["tflops"] = work / (avg / 1e3) / 1e12
-                    e["frac_of_sustained"] = e["tflops"] / (2.0 * pk["bf16_sus"])
+                    e["frac_of_burst"] = e["tflops"] / (f8 * pk["bf16"])
+                    e["frac_of_sustained"] = e["tflops"] / (f8 * pk["bf16_sus"])
                 else:
                     e["gbs"] = work / (avg / 1e3) / 1e9
                     e["frac_of_hbm"] = e["gbs"] / pk["hbm"]
@@ -457,12 +586,14 @@ def run_ours(args, w):
         if bound in ("tensor", "tensor8"):
             ach = work / (avg / 1e3) / 1e12
             f8 = 2.0 if bound == "tensor8" else 1.0
-            roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": f8 * pk["bf16_sus"],
-                    "unit": "TFLOP/s", "frac": ach / (f8 * pk["bf16_sus"]),
-                    "peak_note": (f"bf16 sustained ({pk['src']})" if f8 == 1.0 else
-                                  f"e4m3: 2 x the bf16 sustained ({pk['src']}), the nominal "
+            roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": f8 * tpk,
+                    "unit": "TFLOP/s", "frac": ach / (f8 * tpk),
+                    "peak_note": (f"bf16 {tpk_name} ({pk['src']}): the timed region lasts "
+                                  f"{ms_max / 1e3:.2f} s" if f8 == 1.0 else
+                                  f"e4m3: 2 x the bf16 {tpk_name} ({pk['src']}), the nominal "
                                   "4.5 / 2.25 PF ratio")
-                                 + f"; burst gives frac {ach / (f8 * pk['bf16']):.3f}",
+                                 + f"; frac of the other bf16 peak: "
+                                   f"{ach / (f8 * (pk['bf16_sus'] if burst else pk['bf16'])):.3f}",
                     "traffic": traffic, "algorithmic_per_launch": work}
         else:
             ach = work / (avg / 1e3) / 1e9
@@ -489,19 +620,26 @@ def run_ours(args, w):
                    "kind": "oracle",
                    "sample": f"{reps} x ({rows} of {w.T} rows of {w.name}: full candidate build "
                              f"+ float64 loss and gradients of those rows)"}
+        gemm_ms = sum(kernels[k][1] / kernels[k][0] for k in timed_in_loop)
+        small_ms = sum(kernels[k][1] / kernels[k][0] for k in kernels if k not in timed_in_loop)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "ms_per_step_median": med_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if args.precision == "bf16" else "e4m3 logits GEMM, bf16 gradient GEMMs",
+            "precision": args.precision,
             "data": "synthetic (seeded Zipf targets, N(0,1) x, N(0,1/d) lm_head)",
-            "config": dict(workload_config(w, world), precision=args.precision),
+            "config": workload_config(w, world, dp),
             "step_tflops": step_tflops,
-            "frac_of_bf16_peak": {"sustained": step_tflops / pk["bf16_sus"],
-                                  "burst": step_tflops / pk["bf16"], "datasheet_2250": step_tflops / 2250.0,
-                                  "peaks": pk["src"]},
+            "frac_of_bf16_peak": {"burst": step_tflops / pk["bf16"],
+                                  "sustained": step_tflops / pk["bf16_sus"],
+                                  "datasheet_2250": step_tflops / 2250.0, "peaks": pk["src"]},
             "roofline": roof,
             "kernels": per,
+            "step_breakdown_ms": {"gemms": gemm_ms, "small_kernels": small_ms,
+                                  "step": ms_max / args.steps,
+                                  "outside_kernels": ms_max / args.steps - gemm_ms - small_ms},
             "gpu_launches": launches,
             "clocks": clk,
             "clock_normalized": clock_normalized(step_tflops, per, clk, world),
@@ -510,11 +648,15 @@ def run_ours(args, w):
                                "two gradient GEMMs shrink 2-5x against the full softmax over "
                                "V = 50304 (no hardware stated)",
                 "V_over_P": w.V / w.P,
-                "measured": "profiles/candidate_count_vs_full_softmax.md",
             },
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
+        if dp:
+            line["dp_allreduce"] = {
+                "what": "NCCL all-reduce (sum) of the dense dW [V, d] bf16 after every step, "
+                        "on its own stream, overlapping the next step's build and forward",
+                "bytes": w.V * w.d * 2, "avg_ms": float(np.mean(ar_ms)) if ar_ms else None}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -84,6 +84,15 @@ typedef enum ss_status {
  * per step). */
 SS_API size_t ss_workspace_bytes(int64_t T, int32_t d, int32_t V, int32_t P);
 
+/* Byte offset, inside that workspace, of the gathered rows W_C = lm_head[C]
+ * ([P, d] bf16, row-major, row pitch d) that ss_ce_forward and
+ * ss_ce_forward_e4m3 leave there for the backward (sampled_softmax.py,
+ * SampledSoftmax._gather_rows: a plain row copy, so W_C can be checked bit
+ * for bit against lm_head[C]). Returns (size_t)-1 if the sizes are invalid.
+ * Read-only diagnostics: the rows are valid once the stream has passed the
+ * forward and until the workspace is next used. */
+SS_API size_t ss_workspace_wc_offset(int64_t T, int32_t d, int32_t V, int32_t P);
+
 /* Bytes of workspace ss_build_candidates alone needs for a vocabulary of V
  * classes (0 if V is out of range). ss_workspace_bytes covers it as well. */
 SS_API size_t ss_build_workspace_bytes(int32_t V);
@@ -123,7 +132,9 @@ SS_API ss_status ss_build_candidates(const int32_t* targets, int64_t T, int32_t 
  * GPU that loads the library until the process exits.
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture. All calls on a device share the one array:
+ * before any stream capture. The address is then kept for the life of the
+ * process: after cudaDeviceReset on a device, do not call this entry point
+ * on that device again in the same process. All calls on a device share the one array:
  * calls whose work overlaps on the GPU (two streams, or two host threads
  * without ordering) race and give wrong results, so order them on one
  * stream. Each call rewrites every part of the array it reads, so nothing

@@ -34,6 +34,7 @@ EXPORTS = (
     "ss_status_string", "ss_last_cuda_error", "ss_version", "ss_timing_enable",
     "ss_timing_reset", "ss_timing_count", "ss_timing_query", "ss_prefix_positions",
     "ss_selftest_wait_limit", "ss_ce_forward_e4m3", "ss_workspace_bytes_e4m3", "ss_quantize_e4m3",
+    "ss_workspace_wc_offset",
 )
 
 
@@ -68,6 +69,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     sig = {
         "ss_workspace_bytes": (_sz, [_i64, _i32, _i32, _i32]),
+        "ss_workspace_wc_offset": (_sz, [_i64, _i32, _i32, _i32]),
         "ss_build_workspace_bytes": (_sz, [_i32]),
         "ss_build_candidates": (_i32, [_p, _i64, _i32, _i32, _i64, _i32, _p, _p, _p, _p, _p, _sz, _p]),
         "ss_build_candidates_noalloc": (_i32, [_p, _i64, _i32, _i32, _i64, _i32, _p, _p, _p, _p,
@@ -123,6 +125,12 @@ def _check(fn: str, code: int):
 
 def ss_workspace_bytes(T: int, d: int, V: int, P: int) -> int:
     return int(load().ss_workspace_bytes(T, d, V, P))
+
+
+def ss_workspace_wc_offset(T: int, d: int, V: int, P: int) -> int:
+    """Byte offset of W_C [P, d] bf16 in the workspace after a forward (-1: invalid sizes)."""
+    off = int(load().ss_workspace_wc_offset(T, d, V, P))
+    return -1 if off == (1 << 64) - 1 else off
 
 
 def ss_build_workspace_bytes(V: int) -> int:
@@ -276,10 +284,12 @@ class SampledCE:
         fwd(x, lm_head, self.candidates, self.target_pos, self.T, self.d, self.V, self.P,
             self.loss, self.lse, self.n_valid, self.dev_status, self.workspace, stream)
 
-    def backward(self, grad_loss=None, stream=None):
+    def backward(self, grad_loss=None, stream=None, dW=None):
+        """dx into self.dx; dW into self.dW, or into the [V, d] bf16 tensor `dW`."""
         g = self.grad_loss if grad_loss is None else grad_loss
-        ss_ce_backward(g, self.candidates, self.vocab_pos, self.n_valid, self.T, self.d, self.V, self.P, self.dx, self.dW,
-                       self.dev_status, self.workspace, stream)
+        ss_ce_backward(g, self.candidates, self.vocab_pos, self.n_valid, self.T, self.d, self.V,
+                       self.P, self.dx, self.dW if dW is None else dW, self.dev_status,
+                       self.workspace, stream)
 
     def step(self, targets, x, lm_head, offset, stride=DEFAULT_STRIDE, grad_loss=None, stream=None):
         self.build(targets, offset, stride, stream)

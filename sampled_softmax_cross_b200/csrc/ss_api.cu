@@ -120,13 +120,25 @@ struct TimingState {
 TimingState g_tm;
 constexpr size_t kTimingPairs = 8192;
 
-int timing_begin(const char* name, cudaStream_t s) {
-  if (!g_tm.on || g_tm.used >= kTimingPairs) return -1;
-  if (g_tm.gemms_only && strstr(name, "gemm") == nullptr) return -1;
-  if (g_tm.ev.empty()) {
-    g_tm.ev.resize(2 * kTimingPairs);
-    for (auto& e : g_tm.ev) cudaEventCreate(&e);
+// Events are created when timing is switched on (ss_timing_enable), never
+// inside a launch: creating thousands of events takes the host milliseconds,
+// which inside a timed region would leave the GPU idle.
+cudaError_t timing_make_events() {
+  if (!g_tm.ev.empty()) return cudaSuccess;
+  std::vector<cudaEvent_t> ev(2 * kTimingPairs);
+  for (auto& e : ev) {
+    const cudaError_t r = cudaEventCreate(&e);
+    if (r != cudaSuccess) return r;
   }
+  g_tm.ev.swap(ev);
+  return cudaSuccess;
+}
+
+// `gemm`: the launch is one of the three tensor-core GEMMs (timed also in
+// the GEMMs-only mode).
+int timing_begin(const char* name, bool gemm, cudaStream_t s) {
+  if (!g_tm.on || g_tm.ev.empty() || g_tm.used >= kTimingPairs) return -1;
+  if (g_tm.gemms_only && !gemm) return -1;
   int idx = -1;
   for (size_t i = 0; i < g_tm.names.size(); ++i)
     if (g_tm.names[i] == name) idx = (int)i;
@@ -144,13 +156,15 @@ void timing_end(int slot, cudaStream_t s) {
   if (slot >= 0) cudaEventRecord(g_tm.ev[2 * slot + 1], s);
 }
 
-#define SS_LAUNCH(name, stream, call)                         \
+#define SS_LAUNCH_KIND(name, gemm, stream, call)              \
   do {                                                        \
-    const int _slot = timing_begin(name, stream);             \
+    const int _slot = timing_begin(name, gemm, stream);       \
     cudaError_t _e = (call);                                  \
     timing_end(_slot, stream);                                \
     if (_e != cudaSuccess) return cuda_fail(_e, name);        \
   } while (0)
+#define SS_LAUNCH(name, stream, call) SS_LAUNCH_KIND(name, false, stream, call)
+#define SS_LAUNCH_GEMM(name, stream, call) SS_LAUNCH_KIND(name, true, stream, call)
 
 // -------------------------------------------------------------- workspace --
 constexpr int kBM = 128, kBN = 256, kBMP = 256;  // rows per CTA, cols per tile, rows per pair
@@ -215,6 +229,28 @@ int gcd_int(int64_t a, int64_t b) {
 }
 
 }  // namespace
+
+namespace ssb {
+
+// The two builder launches, shared by ss_build_candidates and
+// ss_build_candidates_noalloc (which differ only in where the bitmap and
+// prefix scratch live). Launch errors go to ss_last_cuda_error and the
+// launches are recorded by the kernel timer like every other launch.
+ss_status enqueue_build(const int32_t* targets, int64_t T, int32_t V, int32_t P, int64_t offset,
+                        int32_t stride, int32_t* candidates, int32_t* target_pos,
+                        int32_t* vocab_pos, int32_t* dev_status, uint32_t* bitmap,
+                        int32_t* prefix, cudaStream_t s) {
+  SS_LAUNCH("build_mark", s,
+            launch_build_mark(targets, T, V, P, offset % V, stride, bitmap, prefix, dev_status, s));
+  SS_LAUNCH("build_emit", s,
+            launch_build_emit(targets, T, V, P, bitmap, prefix, dev_status, candidates, target_pos,
+                              vocab_pos, s));
+  return SS_OK;
+}
+
+ss_status record_cuda_error(cudaError_t e, const char* where) { return cuda_fail(e, where); }
+
+}  // namespace ssb
 
 // ===================================================================== API ==
 // The forward, with the logits GEMM on bf16 operands or (e4m3) on per-tensor
@@ -312,7 +348,7 @@ static ss_status forward_impl(const ss_bf16* x, const ss_bf16* lm_head,
     a.status = kstatus;
     const int tiles = a.tiles_m * a.tiles_n;
     const int kind = e4m3 ? KIND_FWD8 : KIND_FWD;
-    SS_LAUNCH(e4m3 ? "fwd_gemm_ce_e4m3" : "fwd_gemm_ce", s,
+    SS_LAUNCH_GEMM(e4m3 ? "fwd_gemm_ce_e4m3" : "fwd_gemm_ce", s,
               launch_gemm(kind, ta, tb, tc, a, tiles < pairs[kind] ? tiles : pairs[kind], s));
     SS_LAUNCH("row_pass", s, launch_rows(ra, s));
   }
@@ -349,6 +385,11 @@ size_t ss_workspace_bytes(int64_t T, int32_t d, int32_t V, int32_t P) {
   return layout(T, d, V, P).total;
 }
 
+size_t ss_workspace_wc_offset(int64_t T, int32_t d, int32_t V, int32_t P) {
+  if (!sizes_ok(T, d, V, P)) return (size_t)-1;
+  return layout(T, d, V, P).w_c;
+}
+
 size_t ss_build_workspace_bytes(int32_t V) {
   if (V < 1 || V > SS_MAX_VOCAB) return 0;
   return 2 * align_up((size_t)(V + 31) / 32 * 4, 256);
@@ -375,12 +416,8 @@ ss_status ss_build_candidates(const int32_t* targets, int64_t T, int32_t V, int3
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(ws);
   int32_t* prefix = reinterpret_cast<int32_t*>(ws + align_up(nw * 4, 256));
-  SS_LAUNCH("build_mark", s,
-            launch_build_mark(targets, T, V, P, offset % V, stride, bitmap, prefix, dev_status, s));
-  SS_LAUNCH("build_emit", s,
-            launch_build_emit(targets, T, V, P, bitmap, prefix, dev_status, candidates, target_pos,
-                              vocab_pos, s));
-  return SS_OK;
+  return enqueue_build(targets, T, V, P, offset, stride, candidates, target_pos, vocab_pos,
+                       dev_status, bitmap, prefix, s);
 }
 
 ss_status ss_ce_forward(const ss_bf16* x, const ss_bf16* lm_head, const int32_t* candidates,
@@ -475,7 +512,7 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   a.ld_out = d;
   a.status = kstatus;
   const int tiles = a.tiles_m * a.tiles_n;
-  SS_LAUNCH("dx_gemm", s,
+  SS_LAUNCH_GEMM("dx_gemm", s,
             launch_gemm(KIND_DX, ua, wb, dxs, a, tiles < pairs[KIND_DX] ? tiles : pairs[KIND_DX], s));
 
   GemmArgs b{};
@@ -493,7 +530,7 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   b.n_valid = n_valid;
   b.status = kstatus;
   // every resident pair, even without a tile, so that the zero rows are spread over all SMs
-  SS_LAUNCH("dw_gemm_scatter", s, launch_gemm(KIND_DW, ua2, xb, ua2, b, pairs[KIND_DW], s));
+  SS_LAUNCH_GEMM("dw_gemm_scatter", s, launch_gemm(KIND_DW, ua2, xb, ua2, b, pairs[KIND_DW], s));
   return SS_OK;
 }
 
@@ -524,6 +561,7 @@ ss_status ss_selftest_wait_limit(int32_t* dev_status, void* stream) {
 }
 
 ss_status ss_timing_enable(int32_t enable) {
+  if (enable != 0) SS_CUDA(timing_make_events(), "cudaEventCreate");
   g_tm.on = enable != 0;
   g_tm.gemms_only = enable == 2;
   return SS_OK;

@@ -73,4 +73,12 @@ cudaError_t launch_ref_logits_e4m3(const uint8_t* x8, const uint8_t* w8, const i
 cudaError_t launch_zero_rows(uint16_t* dW, int32_t V, int32_t d, const int32_t* vocab_pos,
                              int all_rows, cudaStream_t s);
 
+// Host side (ss_api.cu): the candidate build's two launches on caller-given
+// scratch, and the error record behind ss_last_cuda_error.
+ss_status enqueue_build(const int32_t* targets, int64_t T, int32_t V, int32_t P, int64_t offset,
+                        int32_t stride, int32_t* candidates, int32_t* target_pos,
+                        int32_t* vocab_pos, int32_t* dev_status, uint32_t* bitmap,
+                        int32_t* prefix, cudaStream_t s);
+ss_status record_cuda_error(cudaError_t e, const char* where);
+
 }  // namespace ssb

@@ -36,20 +36,24 @@ uint32_t* g_scratch_ptr[128] = {};
 // Device address of g_build_scratch on the current device. In host code the
 // symbol names a host-side stand-in, not device memory, so the address must
 // come from cudaGetSymbolAddress, once per device, with that device current.
+// The address is kept for the life of the process: a process that destroys
+// the device's primary context (cudaDeviceReset) must not call this entry
+// point on that device again, since the array may then live elsewhere.
 ss_status scratch_for_current_device(uint32_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return SS_ERR_CUDA;
+  if (e != cudaSuccess) return ssb::record_cuda_error(e, "cudaGetDevice");
   if (dev < 0 || dev >= 128) return SS_ERR_UNSUPPORTED_DEVICE;
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_ready[dev]) {
     int major = 0;
     e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    if (e != cudaSuccess) return SS_ERR_CUDA;
+    if (e != cudaSuccess) return ssb::record_cuda_error(e, "cudaDeviceGetAttribute");
     if (major != 10) return SS_ERR_UNSUPPORTED_DEVICE;
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_build_scratch);
-    if (e != cudaSuccess || p == nullptr) return SS_ERR_CUDA;
+    if (e != cudaSuccess) return ssb::record_cuda_error(e, "cudaGetSymbolAddress");
+    if (p == nullptr) return ssb::record_cuda_error(cudaErrorInvalidSymbol, "cudaGetSymbolAddress");
     g_scratch_ptr[dev] = static_cast<uint32_t*>(p);
     g_ready[dev] = true;
   }
@@ -87,11 +91,6 @@ extern "C" SS_API ss_status ss_build_candidates_noalloc(
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint32_t* bitmap = scratch;
   int32_t* prefix = reinterpret_cast<int32_t*>(scratch + kWords);
-  cudaError_t e = ssb::launch_build_mark(targets, T, V, P, offset % V, stride, bitmap, prefix,
-                                         dev_status, s);
-  if (e != cudaSuccess) return SS_ERR_CUDA;
-  e = ssb::launch_build_emit(targets, T, V, P, bitmap, prefix, dev_status, candidates, target_pos,
-                             vocab_pos, s);
-  if (e != cudaSuccess) return SS_ERR_CUDA;
-  return SS_OK;
+  return ssb::enqueue_build(targets, T, V, P, offset, stride, candidates, target_pos, vocab_pos,
+                            dev_status, bitmap, prefix, s);
 }

@@ -50,6 +50,17 @@ def test_status_strings(lib):
     assert capi.ss_version() >= 10000
 
 
+def test_wc_offset_lies_inside_the_workspace(lib):
+    for T, d, V, P in ((512, 128, 50304, 2048), (49152, 768, 50304, 24576), (0, 8, 10, 1),
+                       (700, 200, 3001, 1111)):
+        off = capi.ss_workspace_wc_offset(T, d, V, P)
+        assert off >= 0 and off % 1024 == 0
+        assert off + P * d * 2 <= capi.ss_workspace_bytes(T, d, V, P)
+        assert off + P * d * 2 <= capi.ss_workspace_bytes_e4m3(T, d, V, P) or d % 16
+    assert capi.ss_workspace_wc_offset(512, 127, 50304, 2048) == -1
+    assert capi.ss_workspace_wc_offset(512, 128, 50304, 50305) == -1
+
+
 def test_workspace_bytes_rejects_bad_sizes(lib):
     assert capi.ss_workspace_bytes(512, 128, 50304, 2048) > 0
     assert capi.ss_workspace_bytes(512, 127, 50304, 2048) == 0   # d % 8

@@ -19,8 +19,8 @@ from oracle import sampled_ce as oc
 from sampled_softmax_cross_b200 import capi
 from sampled_softmax_cross_b200 import workloads as wl
 
-from gpu_common import (GRAD_RTOL, LOSS_ATOL, LOSS_RTOL, LSE_ATOL, compare_full, dev_bf16,
-                        rel_fro, run_path)
+from gpu_common import (LOSS_ATOL, LOSS_RTOL, LSE_ATOL, check_grad, compare_full, dev_bf16,
+                        run_path, sample_cols, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -111,10 +111,6 @@ def test_e4m3_rows_with_huge_loss_are_recomputed_exactly():
     compare_full(g, o, t)
 
 
-def _sample(n, k, rng):
-    return np.sort(rng.choice(n, size=min(n, k), replace=False))
-
-
 def test_e4m3_headline_workload():
     w = wl.WORKLOADS["stage2_late"]
     x_bits, lm_bits, t = wl.workload_inputs(w)
@@ -134,15 +130,13 @@ def test_e4m3_headline_workload():
 
     rng = np.random.default_rng(w.seed + 200)
     scale = 1.0 / n
-    rows = _sample(w.T, 256, rng)
+    rows = sample_rows(w.T, 512, rng)
     dx_o = oc.dx_rows(x[rows], w_c, tpos[rows], lse[rows], scale, logit_x_rows=xq[rows],
                       logit_w=wq)
-    dx_g = wl.bits_to_f64(g["dx_bits"][rows])
-    assert rel_fro(dx_g, dx_o) <= GRAD_RTOL, rel_fro(dx_g, dx_o)
-    cols = np.unique(np.concatenate([_sample(w.P, 128, rng), tpos[tpos >= 0][:16]]))
+    check_grad(wl.bits_to_f64(g["dx_bits"][rows]), dx_o, "dx rows")
+    cols = sample_cols(w.P, tpos, 256, rng)
     dw_o = oc.dw_c_rows(x, w_c, tpos, lse, scale, cols, logit_x=xq, logit_w=wq)
-    dw_g = wl.bits_to_f64(g["dW_bits"][cand[cols]])
-    assert rel_fro(dw_g, dw_o) <= GRAD_RTOL, rel_fro(dw_g, dw_o)
+    check_grad(wl.bits_to_f64(g["dW_bits"][cand[cols]]), dw_o, "dW rows")
 
 
 def test_e4m3_empty_microbatch_and_full_vocabulary():

@@ -2,9 +2,12 @@
 
 Small and ragged shapes are compared element by element with a full oracle
 run. The five named workloads are run at full size in the launch
-configuration the benchmark times; their integer outputs are compared in full
-and their floating outputs on all rows (loss, lse) or on seeded samples of
-rows (dX) and of candidate columns (dW), which the oracle computes one by one.
+configuration the benchmark times: their integer outputs are compared in full;
+stage0 (T=16384, P=10240) and the headline stage2_late (T=49152, P=24576) are
+compared in full, every element of dX and dW included; the other two compare
+loss and lse on all rows and dX / dW on rows and candidate columns sampled so
+that every GEMM tile is hit, which the oracle computes one by one. The
+gathered rows W_C are compared with lm_head[C] bit for bit.
 """
 
 import json
@@ -18,8 +21,8 @@ from oracle import sampled_ce as oc
 from sampled_softmax_cross_b200 import capi
 from sampled_softmax_cross_b200 import workloads as wl
 
-from gpu_common import (GRAD_RTOL, LOSS_RTOL, LSE_ATOL, check_build, compare_full, rel_fro,
-                        run_build, run_path)
+from gpu_common import (LOSS_RTOL, LSE_ATOL, check_build, check_grad, compare_full,
+                        dev_bf16, host_bits, run_build, run_path, sample_cols, sample_rows)
 
 pytestmark = pytest.mark.gpu
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -294,12 +297,11 @@ def test_kernel_timing_records_every_kernel():
 
 # ------------------------------------------------ full-size workloads --
 
-def _sample(n, k, rng):
-    return np.sort(rng.choice(n, size=min(n, k), replace=False))
-
-
-@pytest.mark.parametrize("name", ["stage0", "stage2_early", "stage2_late", "full_softmax"])
+@pytest.mark.parametrize("name", ["stage2_early", "stage2_late", "full_softmax"])
 def test_full_size_workload(name):
+    """Full size, the benchmark's launch configuration: integers in full, loss
+    and lse on every row, dX on rows from every M tile, dW on the first and
+    last column of every candidate tile plus random and target columns."""
     w = wl.WORKLOADS[name]
     x_bits, lm_bits, t = wl.workload_inputs(w)
     g = run_path(x_bits, lm_bits, t, w.P, w.offset)
@@ -319,17 +321,55 @@ def test_full_size_workload(name):
 
     rng = np.random.default_rng(w.seed + 100)
     scale = 1.0 / n
-    rows = _sample(w.T, 384, rng)
+    rows = sample_rows(w.T, 768, rng)
     dx_o = oc.dx_rows(x[rows], w_c, tpos[rows], lse[rows], scale)
-    dx_g = wl.bits_to_f64(g["dx_bits"][rows])
-    assert rel_fro(dx_g, dx_o) <= GRAD_RTOL, rel_fro(dx_g, dx_o)
+    check_grad(wl.bits_to_f64(g["dx_bits"][rows]), dx_o, "dx rows")
 
-    cols = np.unique(np.concatenate([_sample(w.P, 256, rng), tpos[tpos >= 0][:32]]))
+    cols = sample_cols(w.P, tpos, 512, rng)
     dw_o = oc.dw_c_rows(x, w_c, tpos, lse, scale, cols)
-    dw_g = wl.bits_to_f64(g["dW_bits"][cand[cols]])
-    assert rel_fro(dw_g, dw_o) <= GRAD_RTOL, rel_fro(dw_g, dw_o)
+    check_grad(wl.bits_to_f64(g["dW_bits"][cand[cols]]), dw_o, "dW rows")
 
     in_c = np.zeros(w.V, bool)
     in_c[cand] = True
     assert np.all(g["dW_bits"][~in_c] == 0)
     assert np.all(g["dx_bits"][tpos < 0] == 0)
+
+
+@pytest.mark.parametrize("name", ["stage0", "stage2_late"])
+def test_full_size_workload_compared_in_full(name):
+    """Every output of a full-size workload against a full float64 oracle run:
+    candidate set and positions bit for bit, loss, lse of every row, and every
+    element of dX and of dW (rows in C; +0.0 bits elsewhere)."""
+    w = wl.WORKLOADS[name]
+    x_bits, lm_bits, t = wl.workload_inputs(w)
+    g = run_path(x_bits, lm_bits, t, w.P, w.offset)
+    o = oracle_run(x_bits, lm_bits, t, w.P, w.offset)
+    compare_full(g, o, t)
+
+
+@pytest.mark.parametrize("name,d", [("tiny", None), ("stage0", None), ("stage2_early", None),
+                                    ("stage2_late", None), ("full_softmax", None),
+                                    ("ragged_d", 200)])
+def test_gathered_rows_are_an_exact_copy(name, d):
+    """W_C = lm_head[C] is a byte copy (SampledSoftmax._gather_rows): the rows the
+    forward leaves in the workspace equal lm_head[C] bit for bit."""
+    if name == "ragged_d":
+        x_bits, lm_bits, t = wl.make_inputs(700, d, 3001, 1.1, 0.05, 41)
+        V, P, off = 3001, 1111, 29
+    else:
+        w = wl.WORKLOADS[name]
+        x_bits, lm_bits, t = wl.workload_inputs(w)
+        V, P, off = w.V, w.P, w.offset
+    T, dd = x_bits.shape
+    for precision in ("bf16", "e4m3") if dd % 16 == 0 else ("bf16",):
+        ce = capi.SampledCE(T, dd, V, P, precision=precision)
+        ce.build(torch.from_numpy(t).cuda(), off)
+        ce.forward(dev_bf16(x_bits), dev_bf16(lm_bits))
+        torch.cuda.synchronize()
+        st = ce.status()
+        assert st[0] == 0 and st[8] == 0, st
+        cand = ce.candidates.cpu().numpy()
+        o0 = capi.ss_workspace_wc_offset(T, dd, V, P)
+        assert o0 >= 0 and o0 % 16 == 0
+        w_c = host_bits(ce.workspace[o0:o0 + P * dd * 2].view(torch.bfloat16).view(P, dd))
+        assert np.array_equal(w_c, lm_bits[cand]), (name, precision)

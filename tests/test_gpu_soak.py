@@ -4,8 +4,10 @@ compute-sanitizer's race checker is not available here, so these look for
 races the way a long training run would meet them: results that change from
 one repetition to the next (the persistent GEMMs' barrier phases wrap many
 times per launch and across launches), or that depend on what another
-stream runs at the same time (the library keeps no state between calls, so
-two workspaces on two streams must not interfere).
+stream runs at the same time (the workspace entry points keep no state
+between calls, so two workspaces on two streams must not interfere; the
+allocation-free build is the one exception, with one scratch array per device
+that every call shares, and is not run on two streams here).
 """
 
 import hashlib

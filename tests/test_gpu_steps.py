@@ -21,7 +21,7 @@ from sampled_softmax_cross_b200 import capi
 from sampled_softmax_cross_b200 import schedule as sc
 from sampled_softmax_cross_b200 import workloads as wl
 
-from gpu_common import (GRAD_RTOL, LOSS_RTOL, LSE_ATOL, compare_full, dev_bf16, rel_fro,
+from gpu_common import (LOSS_RTOL, LSE_ATOL, check_grad, compare_full, dev_bf16,
                         run_build, run_path)
 
 pytestmark = pytest.mark.gpu
@@ -115,7 +115,7 @@ def test_steps_driver_chains_the_sweep_across_counts():
         assert abs(loss - o["loss"]) <= LOSS_RTOL * abs(o["loss"]), (step, loss, o["loss"])
         assert np.max(np.abs(ce.lse[:T].cpu().numpy() - o["lse"])) <= LSE_ATOL
         dx = wl.bits_to_f64(ce.dx[:T].view(torch.int16).cpu().numpy().view(np.uint16))
-        assert rel_fro(dx, o["dx"]) <= GRAD_RTOL
+        check_grad(dx, o["dx"], f"dx step {step}")
         off = o["info"]["next_offset"]
     drv.settle()
     assert drv.sweep.offset == off
