@@ -14,7 +14,9 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libsampled_ce.so")
+# The library to load: the in-tree build, or another build of the same
+# sources named by SAMPLED_CE_LIB (the bounds-checked debug build, say).
+LIB_PATH = os.environ.get("SAMPLED_CE_LIB") or os.path.join(_PKG, "libsampled_ce.so")
 
 DEV_STATUS_WORDS = 16
 DEFAULT_STRIDE = 20011

@@ -25,20 +25,30 @@
 // softmax_ij - [j == t_i] (section "Gradient") and the backward is two plain
 // GEMMs with epilogue scales: dX = (g/n) r (.) (E' W_C), dW_C = (g/n) E'^T x'.
 //
-// Work unit: a 256 x 256 output tile computed by a CTA pair (a cluster of two
-// CTAs on one TPC, tcgen05 cta_group::2). Each CTA loads its own 128 rows of A
+// Work unit: an output tile computed by a CTA pair (a cluster of two CTAs on
+// one TPC, tcgen05 cta_group::2). Each CTA loads its own 128-row block(s) of A
 // and its 128-column half of B; the pair's leader issues M=256, N=256, K=16
 // MMAs that read both CTAs' shared memory and write 128 rows x 256 fp32
-// columns into each CTA's TMEM. Per CTA, persistent over tiles:
-//   warp 0      TMA producer, ring of 32 KB stages (A 128x64 + B 128x64 bf16,
-//               or 128x128 e4m3 codes): 6 in the forward, 5 in the e4m3
-//               forward, 7 in dX and dW
+// columns into each CTA's TMEM.
+//   forward : 256 x 256 tiles, one A block per CTA; two TMEM accumulators let
+//             the epilogue of tile i overlap the MMAs of tile i+1 (12 K blocks
+//             per tile: the epilogue is a large share of a tile's time).
+//   dX, dW  : 512 x 256 tiles, two A blocks per CTA and two MMAs per K step
+//             sharing the B operand, both accumulators for one tile. Per
+//             multiply-add this loads 25% fewer operand bytes from L2 than a
+//             256 x 256 tile: at full clock the operand stream from L2 to the
+//             SMs (about 11 TB/s measured) bounds these GEMMs, not the tensor
+//             cores. Their K loops are hundreds of blocks long, so a
+//             single-buffered accumulator costs under 1%.
+// Per CTA, persistent over tiles:
+//   warp 0      TMA producer, ring of stages (A 128x64 per block + B 128x64
+//               bf16, or 128x128 e4m3 codes): 6 x 32 KB in the forward, 5 in
+//               the e4m3 forward, 4 x 48 KB in dX and dW
 //   warp 1      TMEM owner (2 x 256 columns); in the leader, the MMA issuer
 //               (kind::f16, or kind::f8f6f4 with K=32 for the e4m3 forward)
 //   warps 2..   epilogue, 4 warps (8 in the e4m3 forward, two per TMEM lane
 //               quarter): TMEM -> registers -> math -> global (forward: through
 //               swizzled shared-memory boxes and TMA stores; dX, dW: 16-byte stores)
-// Two TMEM accumulators let the epilogue of tile i overlap the MMAs of i+1.
 #include "sm100.cuh"
 #include "ce_gemm.h"
 #include "sampled_ce.h"
@@ -51,7 +61,6 @@ constexpr int BNH = BN / 2;      // B columns held by each CTA of the pair
 constexpr int BK = 64;
 constexpr int A_STAGE = BM * BK * 2;   // 16 KB
 constexpr int B_STAGE = BNH * BK * 2;  // 16 KB
-constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
 constexpr int EPI_BUF = 32 * 64 * 2;  // one 32-row x 64-column bf16 box (4 KB)
 constexpr int BAR_BYTES = 256;
 constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -66,25 +75,38 @@ constexpr float LOG2E = 1.4426950408889634f;
 // stores -- becomes the longer part: that kind gets two warps per TMEM lane
 // quarter, each taking half of the tile's columns (8% faster measured; the
 // bf16 forward gains nothing from it). dX and dW (hundreds of K blocks per
-// tile) store little, from registers, and use a 7th stage.
+// tile) store little, from registers; their 48 KB stages (two A blocks) fit
+// four times, 192 KB in flight per SM as with seven 32 KB stages.
 template <int KIND>
 struct Op;
 template <>
 struct Op<KIND_FWD> {  // A = x (K-major), B = W_C (K-major)
-  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6, EPI_WARPS = 4;
+  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6, EPI_WARPS = 4, AB = 1;
 };
 template <>
 struct Op<KIND_FWD8> {  // A = x_q, B = W_C,q (e4m3, K-major; 128 per K block)
-  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 5, EPI_WARPS = 8;
+  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 5, EPI_WARPS = 8, AB = 1;
 };
 template <>
 struct Op<KIND_DX> {  // A = E' (K-major), B = W_C viewed [K=P][N=d] (MN-major)
-  static constexpr int A_MN = 0, B_MN = 1, TMA_STORE = 0, STAGES = 7, EPI_WARPS = 4;
+  static constexpr int A_MN = 0, B_MN = 1, TMA_STORE = 0, STAGES = 4, EPI_WARPS = 4, AB = 2;
 };
 template <>
 struct Op<KIND_DW> {  // A = E' viewed [K=T][M=P] (MN-major), B = x' viewed [K=T][N=d] (MN-major)
-  static constexpr int A_MN = 1, B_MN = 1, TMA_STORE = 0, STAGES = 7, EPI_WARPS = 4;
+  static constexpr int A_MN = 1, B_MN = 1, TMA_STORE = 0, STAGES = 4, EPI_WARPS = 4, AB = 2;
 };
+
+// Bytes of one pipeline stage: AB blocks of 128 A rows, and the CTA's half of B.
+template <int KIND>
+constexpr int stage_bytes() {
+  return Op<KIND>::AB * A_STAGE + B_STAGE;
+}
+// Accumulator buffers in TMEM (2 x 256 columns): two tiles in flight when a
+// tile takes one 256-column accumulator, one tile when it takes both.
+template <int KIND>
+constexpr int acc_bufs() {
+  return Op<KIND>::AB == 1 ? 2 : 1;
+}
 
 static_assert(Op<KIND_FWD>::EPI_WARPS / 4 == kFwdSumsPerTileBf16 &&
                   Op<KIND_FWD8>::EPI_WARPS / 4 == kFwdSumsPerTileE4m3,
@@ -101,7 +123,7 @@ constexpr int epi_bytes() {
 }
 template <int KIND>
 constexpr int smem_bytes() {
-  return 1024 + Op<KIND>::STAGES * STAGE_BYTES + epi_bytes<KIND>() + BAR_BYTES;
+  return 1024 + Op<KIND>::STAGES * stage_bytes<KIND>() + epi_bytes<KIND>() + BAR_BYTES;
 }
 static_assert(smem_bytes<KIND_FWD>() <= 232448 && smem_bytes<KIND_FWD8>() <= 232448 &&
                   smem_bytes<KIND_DX>() <= 232448 &&
@@ -170,10 +192,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   constexpr int STAGES = Op<KIND>::STAGES;
+  constexpr int AB = Op<KIND>::AB;             // 128-row A blocks per CTA and tile
+  constexpr int ACC = acc_bufs<KIND>();        // tiles whose accumulators fit in TMEM
+  constexpr int STAGE = stage_bytes<KIND>();
+  constexpr int TILE_ROWS = 2 * BM * AB;       // output rows of a pair's tile
   constexpr bool IS_FWD = KIND == KIND_FWD || KIND == KIND_FWD8;
   constexpr bool F8 = KIND == KIND_FWD8;
   constexpr int BKE = F8 ? 2 * BK : BK;  // K elements per 128-byte row of a stage
-  uint8_t* epi_smem = smem + STAGES * STAGE_BYTES;
+  uint8_t* epi_smem = smem + STAGES * STAGE;
   uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + epi_bytes<KIND>());
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
@@ -191,7 +217,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
       mbar_init(&full[s], 1);   // leader: one expect-tx arrival for both CTAs' bytes
       mbar_init(&empty[s], 1);  // one multicast commit from the leader's MMA
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < ACC; ++a) {
       mbar_init(&tfull[a], 1);   // one multicast commit per finished accumulator
       mbar_init(&tempty[a], 2 * Op<KIND>::EPI_WARPS);  // leader: epilogue warps of both CTAs
     }
@@ -219,7 +245,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
     uint32_t phase = 0;
     bool ok = true;
     for (int tile = cluster; ok && tile < num_tiles; tile += num_clusters) {
-      const int m0 = (tile / args.tiles_n) * (2 * BM) + (int)rank * BM;
+      // A block b of this CTA: rows m0 + b * 2 * BM .. + BM (the pair's
+      // 256-row MMA b takes block b of both CTAs)
+      const int m0 = (tile / args.tiles_n) * TILE_ROWS + (int)rank * BM;
       const int nh0 = (tile % args.tiles_n) * BN + (int)rank * BNH;
       for (int kb = 0; kb < args.num_kb; ++kb) {
         if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, args.status, KIND)) {
@@ -227,16 +255,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
           break;
         }
         if (lane == 0) {
-          uint8_t* sa = smem + stage * STAGE_BYTES;
-          uint8_t* sb = sa + A_STAGE;
+          uint8_t* sa = smem + stage * STAGE;
+          uint8_t* sb = sa + AB * A_STAGE;
           const int k0 = kb * BKE;
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE);
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
-          if (Op<KIND>::A_MN) {
-            tma_load_2d_pair(sa, &tma_a, bar, m0, k0);
-            tma_load_2d_pair(sa + 8192, &tma_a, bar, m0 + 64, k0);
-          } else {
-            tma_load_2d_pair(sa, &tma_a, bar, k0, m0);
+#pragma unroll
+          for (int b = 0; b < AB; ++b) {
+            const int mb = m0 + b * 2 * BM;
+            if (Op<KIND>::A_MN) {
+              tma_load_2d_pair(sa + b * A_STAGE, &tma_a, bar, mb, k0);
+              tma_load_2d_pair(sa + b * A_STAGE + 8192, &tma_a, bar, mb + 64, k0);
+            } else {
+              tma_load_2d_pair(sa + b * A_STAGE, &tma_a, bar, k0, mb);
+            }
           }
           if (Op<KIND>::B_MN) {
             tma_load_2d_pair_hint(sb, &tma_b, bar, nh0, k0, keep_b);
@@ -271,11 +303,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
       int it = 0;
       bool ok = true;
       for (int tile = cluster; ok && tile < num_tiles; tile += num_clusters, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+        const int acc = it % ACC;
+        const uint32_t acc_phase = (it / ACC) & 1;
         if (!warp_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status, KIND)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t d_tmem = tmem_base + acc * AB * BN;  // block b: + b * BN
         for (int kb = 0; kb < args.num_kb; ++kb) {
           if (!warp_wait(&full[stage], phase, abort_flag, args.status, KIND)) {
             ok = false;
@@ -283,18 +315,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
           }
           tc_fence_after();
           if (lane == 0) {
-            const uint32_t a_addr = smem_u32(smem + stage * STAGE_BYTES);
-            const uint32_t b_addr = a_addr + A_STAGE;
+            const uint32_t a_addr = smem_u32(smem + stage * STAGE);
+            const uint32_t b_addr = a_addr + AB * A_STAGE;
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t ad = Op<KIND>::A_MN ? sdesc_sw128(a_addr + kk * 2048, 8192, 1024)
-                                                 : sdesc_sw128(a_addr + kk * 32, 16, 1024);
               const uint64_t bd = Op<KIND>::B_MN ? sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
                                                  : sdesc_sw128(b_addr + kk * 32, 16, 1024);
-              if (F8)  // K = 32 e4m3 per MMA: the same 32 bytes as 16 bf16
-                umma_f8_pair(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
-              else
-                umma_bf16_pair(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+#pragma unroll
+              for (int b = 0; b < AB; ++b) {
+                const uint32_t ab = a_addr + b * A_STAGE;
+                const uint64_t ad = Op<KIND>::A_MN ? sdesc_sw128(ab + kk * 2048, 8192, 1024)
+                                                   : sdesc_sw128(ab + kk * 32, 16, 1024);
+                if (F8)  // K = 32 e4m3 per MMA: the same 32 bytes as 16 bf16
+                  umma_f8_pair(d_tmem + b * BN, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                else
+                  umma_bf16_pair(d_tmem + b * BN, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+              }
             }
             umma_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
           }
@@ -349,29 +385,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
       }
     }
     for (int tile = cluster; tile < num_tiles; tile += num_clusters, ++it) {
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+      const int acc = it % ACC;
+      const uint32_t acc_phase = (it / ACC) & 1;
       const int m_blk = tile / args.tiles_n, n_blk = tile % args.tiles_n;
-      const int m0 = m_blk * (2 * BM) + (int)rank * BM, n0 = n_blk * BN;
-      const int row = m0 + q * 32 + lane;
-      const bool row_ok = row < args.M;
+      const int n0 = n_blk * BN;
+      // this lane's row in A block b is row0 + b * 2 * BM
+      const int row0 = m_blk * TILE_ROWS + (int)rank * BM + q * 32 + lane;
 
       // per-row values, loaded before the accumulator is ready
       float ref2 = 0.f;  // forward: ref_i * log2(e)
       bool keep = true;  // forward: store E (false on ignored rows: store 0)
-      float rs = scale;  // dX: (g / n) * r_i
-      int32_t cls = -1;
-      if (IS_FWD && row_ok) {
-        ref2 = __ldg(args.ref + row) * LOG2E;
-        keep = __ldg(args.tpos + row) >= 0;
+      // dX: (g / n) * r_i and dW: the row's class id, for A blocks 0 and 1
+      float rs0 = scale, rs1 = scale;
+      int32_t cls0 = -1, cls1 = -1;
+      if (IS_FWD && row0 < args.M) {
+        ref2 = __ldg(args.ref + row0) * LOG2E;
+        keep = __ldg(args.tpos + row0) >= 0;
       }
-      if (KIND == KIND_DX) rs = row_ok ? scale * __ldg(args.rscale + row) : 0.f;
-      if (KIND == KIND_DW && row_ok) cls = __ldg(args.cand + row);
+      if (KIND == KIND_DX) {
+        rs0 = row0 < args.M ? scale * __ldg(args.rscale + row0) : 0.f;
+        if (AB > 1) rs1 = row0 + 2 * BM < args.M ? scale * __ldg(args.rscale + row0 + 2 * BM) : 0.f;
+      }
+      if (KIND == KIND_DW) {
+        if (row0 < args.M) cls0 = __ldg(args.cand + row0);
+        if (AB > 1 && row0 + 2 * BM < args.M) cls1 = __ldg(args.cand + row0 + 2 * BM);
+      }
 
       if (!warp_wait(&tfull[acc], acc_phase, abort_flag, args.status, KIND)) break;
       tc_fence_after();
 
-      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const int n_chunks = min(BN / 64, (args.N - n0 + 63) / 64);  // with valid columns
       const int c_end = min(c_begin + CPW, n_chunks);
       float s_tile = 0.f;
@@ -381,117 +423,129 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
         if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
       }
 
-      for (int c = c_begin; c < c_end; ++c) {
-        const int col0 = n0 + c * 64;
-        uint32_t r0[32], r1[32];
-        tmem_ld32(t_row + c * 64, r0);
-        tmem_ld32(t_row + c * 64 + 32, r1);
-        tmem_wait_ld();
-        if (c == c_end - 1) {
-          // all TMEM reads of this accumulator are done: hand it back to the leader
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
-        }
-        float v[64];
+#pragma unroll 1
+      for (int b = 0; b < AB; ++b) {
+        const int row = row0 + b * 2 * BM;
+        const bool row_ok = row < args.M;
+        const float rs = b == 0 ? rs0 : rs1;
+        const int32_t cl = b == 0 ? cls0 : cls1;
+        const uint32_t t_row =
+            tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((acc * AB + b) * BN);
+        for (int c = c_begin; c < c_end; ++c) {
+          const int col0 = n0 + c * 64;
+          uint32_t r0[32], r1[32];
+          tmem_ld32(t_row + c * 64, r0);
+          tmem_ld32(t_row + c * 64 + 32, r1);
+          tmem_wait_ld();
+          if (b == AB - 1 && c == c_end - 1) {
+            // all TMEM reads of this accumulator are done: hand it back to the leader
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+          }
+          float v[64];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          v[j] = __uint_as_float(r0[j]);
-          v[32 + j] = __uint_as_float(r1[j]);
-        }
+          for (int j = 0; j < 32; ++j) {
+            v[j] = __uint_as_float(r0[j]);
+            v[32 + j] = __uint_as_float(r1[j]);
+          }
 
-        if (IS_FWD) {
-          // E = exp(z - ref) and its row sum over the tile's valid columns
-          const int nvalid = min(64, args.N - col0);
-          float sp[8];  // independent partial sums (short dependency chains)
+          if (IS_FWD) {
+            // E = exp(z - ref) and its row sum over the tile's valid columns
+            const int nvalid = min(64, args.N - col0);
+            float sp[8];  // independent partial sums (short dependency chains)
 #pragma unroll
-          for (int u = 0; u < 8; ++u) sp[u] = 0.f;
-          if (nvalid == 64) {
+            for (int u = 0; u < 8; ++u) sp[u] = 0.f;
+            if (nvalid == 64) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-              v[j] = ex2_approx(fmaf(v[j], zs, -ref2));
-              sp[j & 7] += v[j];
-            }
-          } else {
+              for (int j = 0; j < 64; ++j) {
+                v[j] = ex2_approx(fmaf(v[j], zs, -ref2));
+                sp[j & 7] += v[j];
+              }
+            } else {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-              v[j] = j < nvalid ? ex2_approx(fmaf(v[j], zs, -ref2)) : 0.f;
-              sp[j & 7] += v[j];
-            }
-          }
-          s_tile += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-          if (!keep) {
-#pragma unroll
-            for (int j = 0; j < 64; ++j) v[j] = 0.f;
-          }
-        } else if (KIND == KIND_DX) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) v[j] *= rs;
-        } else {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) v[j] *= scale;
-        }
-
-        if (Op<KIND>::TMA_STORE) {
-          // bf16 tile -> swizzled staging box -> TMA store
-          uint8_t* buf = epi_smem + (e * 2 + (store_ctr & 1)) * EPI_BUF;
-          if (lane == 0) bulk_wait_read<1>();
-          __syncwarp();
-          const uint32_t base = smem_u32(buf) + lane * 128;
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            st_shared_v4(base + ((cc ^ (lane & 7)) << 4), pack_bf16x2(v[cc * 8 + 0], v[cc * 8 + 1]),
-                         pack_bf16x2(v[cc * 8 + 2], v[cc * 8 + 3]),
-                         pack_bf16x2(v[cc * 8 + 4], v[cc * 8 + 5]),
-                         pack_bf16x2(v[cc * 8 + 6], v[cc * 8 + 7]));
-          }
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0 && m0 + q * 32 < args.M) {
-            if (IS_FWD)
-              tma_store_2d_hint(&tma_c, buf, col0, m0 + q * 32, store_policy);
-            else
-              tma_store_2d(&tma_c, buf, col0, m0 + q * 32);
-            bulk_commit();
-          }
-          ++store_ctr;
-        } else if (KIND != KIND_DW) {
-          // bf16 row segment straight from registers (16-byte stores)
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(args.out + (size_t)row * args.ld_out + col0);
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-              if (col0 + cc * 8 < args.N) {
-                const uint4 w = make_uint4(pack_bf16x2(v[cc * 8 + 0], v[cc * 8 + 1]),
-                                           pack_bf16x2(v[cc * 8 + 2], v[cc * 8 + 3]),
-                                           pack_bf16x2(v[cc * 8 + 4], v[cc * 8 + 5]),
-                                           pack_bf16x2(v[cc * 8 + 6], v[cc * 8 + 7]));
-                if (IS_FWD)
-                  __stcs(dst + cc, w);  // E is a write-once stream: do not keep it in L2
-                else
-                  dst[cc] = w;
+              for (int j = 0; j < 64; ++j) {
+                v[j] = j < nvalid ? ex2_approx(fmaf(v[j], zs, -ref2)) : 0.f;
+                sp[j & 7] += v[j];
               }
             }
+            s_tile += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+            if (!keep) {
+#pragma unroll
+              for (int j = 0; j < 64; ++j) v[j] = 0.f;
+            }
+          } else if (KIND == KIND_DX) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) v[j] *= rs;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) v[j] *= scale;
           }
-        } else {  // KIND_DW: row `row` of dW_C goes to row cand[row] of dW
-          if (row_ok && cls >= 0 && cls < args.V) {
-            uint4* dst = reinterpret_cast<uint4*>(args.dW + (size_t)cls * args.N + col0);
+
+          if (Op<KIND>::TMA_STORE) {
+            // bf16 tile -> swizzled staging box -> TMA store
+            uint8_t* buf = epi_smem + (e * 2 + (store_ctr & 1)) * EPI_BUF;
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            const uint32_t base = smem_u32(buf) + lane * 128;
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc) {
-              if (col0 + cc * 8 < args.N) {
-                uint4 w;
-                w.x = pack_bf16x2(v[cc * 8 + 0], v[cc * 8 + 1]);
-                w.y = pack_bf16x2(v[cc * 8 + 2], v[cc * 8 + 3]);
-                w.z = pack_bf16x2(v[cc * 8 + 4], v[cc * 8 + 5]);
-                w.w = pack_bf16x2(v[cc * 8 + 6], v[cc * 8 + 7]);
-                dst[cc] = w;
+              st_shared_v4(base + ((cc ^ (lane & 7)) << 4),
+                           pack_bf16x2(v[cc * 8 + 0], v[cc * 8 + 1]),
+                           pack_bf16x2(v[cc * 8 + 2], v[cc * 8 + 3]),
+                           pack_bf16x2(v[cc * 8 + 4], v[cc * 8 + 5]),
+                           pack_bf16x2(v[cc * 8 + 6], v[cc * 8 + 7]));
+            }
+            fence_async_smem();
+            __syncwarp();
+            const int box_row = row - lane;  // first row of this warp's 32-row box
+            if (lane == 0 && box_row < args.M) {
+              if (IS_FWD)
+                tma_store_2d_hint(&tma_c, buf, col0, box_row, store_policy);
+              else
+                tma_store_2d(&tma_c, buf, col0, box_row);
+              bulk_commit();
+            }
+            ++store_ctr;
+          } else if (KIND != KIND_DW) {
+            // bf16 row segment straight from registers (16-byte stores)
+            if (row_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(args.out + (size_t)row * args.ld_out + col0);
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) {
+                if (col0 + cc * 8 < args.N) {
+                  const uint4 w = make_uint4(pack_bf16x2(v[cc * 8 + 0], v[cc * 8 + 1]),
+                                             pack_bf16x2(v[cc * 8 + 2], v[cc * 8 + 3]),
+                                             pack_bf16x2(v[cc * 8 + 4], v[cc * 8 + 5]),
+                                             pack_bf16x2(v[cc * 8 + 6], v[cc * 8 + 7]));
+                  if (IS_FWD)
+                    __stcs(dst + cc, w);  // E is a write-once stream: do not keep it in L2
+                  else
+                    dst[cc] = w;
+                }
+              }
+            }
+          } else {  // KIND_DW: row `row` of dW_C goes to row cand[row] of dW
+            if (row_ok && cl >= 0 && cl < args.V) {
+              uint4* dst = reinterpret_cast<uint4*>(args.dW + (size_t)cl * args.N + col0);
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) {
+                if (col0 + cc * 8 < args.N) {
+                  uint4 w;
+                  w.x = pack_bf16x2(v[cc * 8 + 0], v[cc * 8 + 1]);
+                  w.y = pack_bf16x2(v[cc * 8 + 2], v[cc * 8 + 3]);
+                  w.z = pack_bf16x2(v[cc * 8 + 4], v[cc * 8 + 5]);
+                  w.w = pack_bf16x2(v[cc * 8 + 6], v[cc * 8 + 7]);
+                  dst[cc] = w;
+                }
               }
             }
           }
         }
       }
 
-      if (IS_FWD && row_ok) args.rowsum[(size_t)(n_blk * HALVES + half) * args.M + row] = s_tile;
+      if (IS_FWD && row0 < args.M)
+        args.rowsum[(size_t)(n_blk * HALVES + half) * args.M + row0] = s_tile;
     }
     if (lane == 0) bulk_wait<0>();
     __syncwarp();
@@ -511,6 +565,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+int gemm_tile_rows(int kind) {
+  switch (kind) {
+    case KIND_FWD: return 2 * BM * Op<KIND_FWD>::AB;
+    case KIND_FWD8: return 2 * BM * Op<KIND_FWD8>::AB;
+    case KIND_DX: return 2 * BM * Op<KIND_DX>::AB;
+    default: return 2 * BM * Op<KIND_DW>::AB;
   }
 }
 

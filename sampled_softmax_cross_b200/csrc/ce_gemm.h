@@ -16,7 +16,7 @@ constexpr int kFwdSumsPerTileBf16 = 1, kFwdSumsPerTileE4m3 = 2;
 // Arguments of the three tcgen05 GEMMs (forward logits, dX, dW_C).
 struct GemmArgs {
   int32_t M, N, K;           // output rows, output cols, contraction length
-  int32_t tiles_m, tiles_n;  // ceil(M / 256) (CTA-pair rows), ceil(N / 256)
+  int32_t tiles_m, tiles_n;  // ceil(M / gemm_tile_rows(kind)), ceil(N / 256)
   int32_t num_kb;            // K blocks: ceil(K / 64), ceil(K / 128) for e4m3
   // forward epilogue: E = exp(z - ref) and its per-tile row sums
   const int32_t* tpos;  // [M] target position of each row, -1 = ignored
@@ -47,6 +47,9 @@ constexpr int kNumGemmKinds = 4;
 cudaError_t launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& c, const GemmArgs& args, int pairs, cudaStream_t s);
 int gemm_smem_bytes(int kind);
+// Output rows of one CTA pair's tile (256, or 512 where a tile takes two
+// 128-row A blocks per CTA); GemmArgs::tiles_m counts tiles of this height.
+int gemm_tile_rows(int kind);
 const void* gemm_kernel_ptr(int kind);
 int gemm_max_pairs(int kind, int sms);
 // One CTA that runs the pipelines' bounded wait out on purpose (ce_gemm.cu).

@@ -167,7 +167,7 @@ void timing_end(int slot, cudaStream_t s) {
 #define SS_LAUNCH_GEMM(name, stream, call) SS_LAUNCH_KIND(name, true, stream, call)
 
 // -------------------------------------------------------------- workspace --
-constexpr int kBM = 128, kBN = 256, kBMP = 256;  // rows per CTA, cols per tile, rows per pair
+constexpr int kBM = 128, kBN = 256;  // A rows per TMA box, output columns per tile
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -336,7 +336,8 @@ static ss_status forward_impl(const ss_bf16* x, const ss_bf16* lm_head,
     a.M = (int32_t)T;
     a.N = P;
     a.K = d;
-    a.tiles_m = (int32_t)((T + kBMP - 1) / kBMP);
+    const int kind = e4m3 ? KIND_FWD8 : KIND_FWD;
+    a.tiles_m = (int32_t)((T + gemm_tile_rows(kind) - 1) / gemm_tile_rows(kind));
     a.tiles_n = L.tiles_n;
     a.num_kb = e4m3 ? (d + 127) / 128 : (d + 63) / 64;
     a.tpos = target_pos;
@@ -347,7 +348,6 @@ static ss_status forward_impl(const ss_bf16* x, const ss_bf16* lm_head,
     a.ld_out = L.ldz;
     a.status = kstatus;
     const int tiles = a.tiles_m * a.tiles_n;
-    const int kind = e4m3 ? KIND_FWD8 : KIND_FWD;
     SS_LAUNCH_GEMM(e4m3 ? "fwd_gemm_ce_e4m3" : "fwd_gemm_ce", s,
               launch_gemm(kind, ta, tb, tc, a, tiles < pairs[kind] ? tiles : pairs[kind], s));
     SS_LAUNCH("row_pass", s, launch_rows(ra, s));
@@ -502,7 +502,7 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   a.M = (int32_t)T;
   a.N = d;
   a.K = P;
-  a.tiles_m = (int32_t)((T + kBMP - 1) / kBMP);
+  a.tiles_m = (int32_t)((T + gemm_tile_rows(KIND_DX) - 1) / gemm_tile_rows(KIND_DX));
   a.tiles_n = (d + kBN - 1) / kBN;
   a.num_kb = (P + 63) / 64;
   a.grad_loss = grad_loss;
@@ -519,7 +519,7 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   b.M = P;
   b.N = d;
   b.K = (int32_t)T;
-  b.tiles_m = (P + kBMP - 1) / kBMP;
+  b.tiles_m = (P + gemm_tile_rows(KIND_DW) - 1) / gemm_tile_rows(KIND_DW);
   b.tiles_n = (d + kBN - 1) / kBN;
   b.num_kb = (int32_t)((T + 63) / 64);
   b.cand = candidates;
