@@ -4,6 +4,12 @@
 the C-ABI library from ``csrc/``; it rebuilds only when a source is newer than
 the library. The CUDA runtime is linked statically, so the library needs only
 the NVIDIA driver at run time.
+
+``build(bounds_check=True)`` (``--bounds``) builds the same sources with
+SS_BOUNDS_CHECK=1 into ``libsampled_ce_bounds.so``: the kernels check the
+indices they compute before each guarded access and record SS_ERR_BAD_INDEX
+(detail 200 + site) in the status words instead of touching memory out of
+range. Load it with SAMPLED_CE_LIB=<path> (the binding reads that variable).
 """
 
 from __future__ import annotations
@@ -18,6 +24,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsampled_ce.so")
+LIB_BOUNDS = os.path.join(PKG, "libsampled_ce_bounds.so")
 SOURCES = ["ss_api.cu", "ce_kernels.cu", "ce_gemm.cu", "ss_noalloc.cu"]
 HEADERS = ["sm100.cuh", "ss_internal.h", "ce_gemm.h"]
 
@@ -43,38 +50,46 @@ def _inputs():
     return files
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not force and not ptxas_info and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          bounds_check: bool = False) -> str:
+    lib = LIB_BOUNDS if bounds_check else LIB
+    if not force and not ptxas_info and up_to_date(lib):
+        return lib
     objs = []
-    build_dir = os.path.join(PKG, "_build")
+    build_dir = os.path.join(PKG, "_build_bounds" if bounds_check else "_build")
     os.makedirs(build_dir, exist_ok=True)
+    procs = []
     for src in SOURCES:
         obj = os.path.join(build_dir, src.replace(".cu", ".o"))
         cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-c", os.path.join(CSRC, src), "-o", obj]
+        if bounds_check:
+            cmd[1:1] = ["-DSS_BOUNDS_CHECK=1"]
         if ptxas_info:
             cmd[1:1] = ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+        procs.append((cmd, subprocess.Popen(cmd)))
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    for cmd, p in procs:
+        if p.wait() != 0:
+            raise subprocess.CalledProcessError(p.returncode, cmd)
+    tmp = lib + ".tmp"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
            "-Xcompiler", "-fPIC", "-lcudart_static", "-ldl", "-lpthread", "-lrt"]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas" in sys.argv,
+                bounds_check="--bounds" in sys.argv))

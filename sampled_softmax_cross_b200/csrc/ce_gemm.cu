@@ -81,19 +81,23 @@ template <int KIND>
 struct Op;
 template <>
 struct Op<KIND_FWD> {  // A = x (K-major), B = W_C (K-major)
-  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6, EPI_WARPS = 4, AB = 1;
+  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6, EPI_WARPS = 4, AB = 1,
+                       EPI_BUFS = 2;
 };
 template <>
 struct Op<KIND_FWD8> {  // A = x_q, B = W_C,q (e4m3, K-major; 128 per K block)
-  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 5, EPI_WARPS = 8, AB = 1;
+  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 5, EPI_WARPS = 8, AB = 1,
+                       EPI_BUFS = 2;
 };
 template <>
 struct Op<KIND_DX> {  // A = E' (K-major), B = W_C viewed [K=P][N=d] (MN-major)
-  static constexpr int A_MN = 0, B_MN = 1, TMA_STORE = 0, STAGES = 4, EPI_WARPS = 4, AB = 2;
+  static constexpr int A_MN = 0, B_MN = 1, TMA_STORE = 0, STAGES = 4, EPI_WARPS = 4, AB = 2,
+                       EPI_BUFS = 0;
 };
 template <>
 struct Op<KIND_DW> {  // A = E' viewed [K=T][M=P] (MN-major), B = x' viewed [K=T][N=d] (MN-major)
-  static constexpr int A_MN = 1, B_MN = 1, TMA_STORE = 0, STAGES = 4, EPI_WARPS = 4, AB = 2;
+  static constexpr int A_MN = 1, B_MN = 1, TMA_STORE = 0, STAGES = 4, EPI_WARPS = 4, AB = 2,
+                       EPI_BUFS = 0;
 };
 
 // Bytes of one pipeline stage: AB blocks of 128 A rows, and the CTA's half of B.
@@ -119,7 +123,7 @@ constexpr int num_threads() {
 }
 template <int KIND>
 constexpr int epi_bytes() {
-  return Op<KIND>::TMA_STORE ? Op<KIND>::EPI_WARPS * 2 * EPI_BUF : 0;
+  return Op<KIND>::TMA_STORE ? Op<KIND>::EPI_WARPS * Op<KIND>::EPI_BUFS * EPI_BUF : 0;
 }
 template <int KIND>
 constexpr int smem_bytes() {
@@ -258,23 +262,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
           uint8_t* sa = smem + stage * STAGE;
           uint8_t* sb = sa + AB * A_STAGE;
           const int k0 = kb * BKE;
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE);
-          const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+          // a TMA box must start on a 16-byte boundary of its inner dimension
+          // (a failed check skips the loads; the pipeline then times out)
+          const bool aligned = SS_CHECK((k0 * (F8 ? 1 : 2)) % 16 == 0, args.status, 9);
+          if (aligned && rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE);
+          if (aligned) {
+            const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
 #pragma unroll
-          for (int b = 0; b < AB; ++b) {
-            const int mb = m0 + b * 2 * BM;
-            if (Op<KIND>::A_MN) {
-              tma_load_2d_pair(sa + b * A_STAGE, &tma_a, bar, mb, k0);
-              tma_load_2d_pair(sa + b * A_STAGE + 8192, &tma_a, bar, mb + 64, k0);
-            } else {
-              tma_load_2d_pair(sa + b * A_STAGE, &tma_a, bar, k0, mb);
+            for (int b = 0; b < AB; ++b) {
+              const int mb = m0 + b * 2 * BM;
+              if (Op<KIND>::A_MN) {
+                tma_load_2d_pair(sa + b * A_STAGE, &tma_a, bar, mb, k0);
+                tma_load_2d_pair(sa + b * A_STAGE + 8192, &tma_a, bar, mb + 64, k0);
+              } else {
+                tma_load_2d_pair(sa + b * A_STAGE, &tma_a, bar, k0, mb);
+              }
             }
-          }
-          if (Op<KIND>::B_MN) {
-            tma_load_2d_pair_hint(sb, &tma_b, bar, nh0, k0, keep_b);
-            tma_load_2d_pair_hint(sb + 8192, &tma_b, bar, nh0 + 64, k0, keep_b);
-          } else {
-            tma_load_2d_pair_hint(sb, &tma_b, bar, k0, nh0, keep_b);
+            if (Op<KIND>::B_MN) {
+              tma_load_2d_pair_hint(sb, &tma_b, bar, nh0, k0, keep_b);
+              tma_load_2d_pair_hint(sb + 8192, &tma_b, bar, nh0 + 64, k0, keep_b);
+            } else {
+              tma_load_2d_pair_hint(sb, &tma_b, bar, k0, nh0, keep_b);
+            }
           }
         }
         __syncwarp();
@@ -393,14 +402,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
       const int row0 = m_blk * TILE_ROWS + (int)rank * BM + q * 32 + lane;
 
       // per-row values, loaded before the accumulator is ready
-      float ref2 = 0.f;  // forward: ref_i * log2(e)
-      bool keep = true;  // forward: store E (false on ignored rows: store 0)
+      // forward: ref_i * log2(e), and whether E is stored (0 on ignored rows),
+      // for A blocks 0 and 1
+      float ref2_0 = 0.f, ref2_1 = 0.f;
+      bool keep0 = true, keep1 = true;
       // dX: (g / n) * r_i and dW: the row's class id, for A blocks 0 and 1
       float rs0 = scale, rs1 = scale;
       int32_t cls0 = -1, cls1 = -1;
       if (IS_FWD && row0 < args.M) {
-        ref2 = __ldg(args.ref + row0) * LOG2E;
-        keep = __ldg(args.tpos + row0) >= 0;
+        ref2_0 = __ldg(args.ref + row0) * LOG2E;
+        keep0 = __ldg(args.tpos + row0) >= 0;
+      }
+      if (IS_FWD && AB > 1 && row0 + 2 * BM < args.M) {
+        ref2_1 = __ldg(args.ref + row0 + 2 * BM) * LOG2E;
+        keep1 = __ldg(args.tpos + row0 + 2 * BM) >= 0;
       }
       if (KIND == KIND_DX) {
         rs0 = row0 < args.M ? scale * __ldg(args.rscale + row0) : 0.f;
@@ -416,7 +431,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
 
       const int n_chunks = min(BN / 64, (args.N - n0 + 63) / 64);  // with valid columns
       const int c_end = min(c_begin + CPW, n_chunks);
-      float s_tile = 0.f;
       if (c_begin >= c_end) {  // no valid column of this tile for this warp
         tc_fence_before();
         __syncwarp();
@@ -429,8 +443,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
         const bool row_ok = row < args.M;
         const float rs = b == 0 ? rs0 : rs1;
         const int32_t cl = b == 0 ? cls0 : cls1;
+        const float ref2 = b == 0 ? ref2_0 : ref2_1;
+        const bool keep = b == 0 ? keep0 : keep1;
+        float s_tile = 0.f;
         const uint32_t t_row =
             tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((acc * AB + b) * BN);
+        if (!SS_CHECK((acc * AB + b + 1) * BN <= (int)TMEM_COLS, args.status, 8)) continue;
         for (int c = c_begin; c < c_end; ++c) {
           const int col0 = n0 + c * 64;
           uint32_t r0[32], r1[32];
@@ -484,8 +502,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
 
           if (Op<KIND>::TMA_STORE) {
             // bf16 tile -> swizzled staging box -> TMA store
-            uint8_t* buf = epi_smem + (e * 2 + (store_ctr & 1)) * EPI_BUF;
-            if (lane == 0) bulk_wait_read<1>();
+            constexpr int NB = Op<KIND>::EPI_BUFS > 0 ? Op<KIND>::EPI_BUFS : 1;
+            uint8_t* buf = epi_smem + (e * NB + (int)(store_ctr % NB)) * EPI_BUF;
+            if (lane == 0) bulk_wait_read<NB - 1>();  // this buffer's last store has read it
             __syncwarp();
             const uint32_t base = smem_u32(buf) + lane * 128;
 #pragma unroll
@@ -526,6 +545,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
               }
             }
           } else {  // KIND_DW: row `row` of dW_C goes to row cand[row] of dW
+            if (row_ok && !(cl >= 0 && cl < args.V)) (void)SS_CHECK(false, args.status, 7);
             if (row_ok && cl >= 0 && cl < args.V) {
               uint4* dst = reinterpret_cast<uint4*>(args.dW + (size_t)cl * args.N + col0);
 #pragma unroll
@@ -542,10 +562,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
             }
           }
         }
+        if (IS_FWD && row_ok) args.rowsum[(size_t)(n_blk * HALVES + half) * args.M + row] = s_tile;
       }
-
-      if (IS_FWD && row0 < args.M)
-        args.rowsum[(size_t)(n_blk * HALVES + half) * args.M + row0] = s_tile;
     }
     if (lane == 0) bulk_wait<0>();
     __syncwarp();

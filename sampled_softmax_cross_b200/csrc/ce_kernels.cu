@@ -250,7 +250,7 @@ __global__ void __cluster_dims__(kBuildCluster, 1, 1) __launch_bounds__(kBuildTh
 // candidates / vocab_pos from the bitmap (threads [0, V)), target_pos (threads [V, V+T)).
 __global__ void k_build_emit(const int32_t* __restrict__ targets, int64_t T, int32_t V, int32_t P,
                              const uint32_t* __restrict__ bitmap, const int32_t* __restrict__ prefix,
-                             const int32_t* __restrict__ st, int32_t* __restrict__ candidates,
+                             int32_t* __restrict__ st, int32_t* __restrict__ candidates,
                              int32_t* __restrict__ target_pos, int32_t* __restrict__ vocab_pos) {
   const int code = *reinterpret_cast<const volatile int32_t*>(st);
   const int64_t n = (int64_t)V + T;
@@ -268,7 +268,7 @@ __global__ void k_build_emit(const int32_t* __restrict__ targets, int64_t T, int
       if ((bits >> b) & 1u) {
         const int pos = prefix[c >> 5] + __popc(bits & ((1u << b) - 1u));
         vocab_pos[c] = pos;
-        candidates[pos] = c;
+        if (SS_CHECK(pos >= 0 && pos < P, st + 8, 1)) candidates[pos] = c;
       } else {
         vocab_pos[c] = -1;
       }
@@ -281,7 +281,8 @@ __global__ void k_build_emit(const int32_t* __restrict__ targets, int64_t T, int
       }
       const uint32_t bits = bitmap[t >> 5];
       const int b = t & 31;
-      target_pos[i] = prefix[t >> 5] + __popc(bits & ((1u << b) - 1u));
+      const int pos = prefix[t >> 5] + __popc(bits & ((1u << b) - 1u));
+      target_pos[i] = SS_CHECK(((bits >> b) & 1u) && pos < P, st + 8, 2) ? pos : -1;
     }
   }
 }
@@ -587,12 +588,16 @@ __global__ void __launch_bounds__(256, 3) k_rows(RowArgs a) {
     const bool fix = in && !(S < kFixThreshold);  // overflow (or NaN): exact recomputation later
     const float rs = (in && valid && !fix) ? 1.f / S : 0.f;
     if (lane < 8) {
-      if (in && fix) a.fix_list[atomicAdd(a.fix_count, 1)] = (int32_t)r;
+      if (in && fix) {
+        const int k = atomicAdd(a.fix_count, 1);
+        if (SS_CHECK(k < a.T, a.status, 3)) a.fix_list[k] = (int32_t)r;
+      }
       if (in && !fix) {
         a.lse[r] = __ldg(a.ref + r) + logf(S);
         a.loss_rows[r] = valid ? logf(S) : 0.f;
         a.rscale[r] = rs;
-        if (valid) a.u[r * a.ldz + tp] = (uint16_t)(pack_bf16x2(1.f - S, 0.f) & 0xffffu);
+        if (valid && SS_CHECK(tp < a.ldz, a.status, 4))
+          a.u[r * a.ldz + tp] = (uint16_t)(pack_bf16x2(1.f - S, 0.f) & 0xffffu);
       }
     }
     {  // loss sum and valid count of the warp's 8 rows, fixed order
@@ -703,11 +708,13 @@ __global__ void __launch_bounds__(kFinThreads) k_finalize(RowArgs a, int32_t npa
   __shared__ float sh[33];
   __shared__ float s_zt;
   __shared__ double s_sum[32], s_cnt[32];
-  const int n = *reinterpret_cast<volatile int32_t*>(a.fix_count);
+  int n = *reinterpret_cast<volatile int32_t*>(a.fix_count);
+  if (!SS_CHECK(n <= a.T, a.status, 5)) n = 0;
   const int vpr = a.d / 8;
   const int nt = blockDim.x;
   for (int k = 0; k < n; ++k) {
     const int64_t r = a.fix_list[k];
+    if (!SS_CHECK(r >= 0 && r < a.T, a.status, 6)) continue;
     const int tp = a.tpos[r];
     const bool valid = tp >= 0 && tp < a.P;
     const uint4* xr = reinterpret_cast<const uint4*>(a.x) + r * vpr;
@@ -874,7 +881,7 @@ cudaError_t launch_build_mark(const int32_t* targets, int64_t T, int32_t V, int3
 
 cudaError_t launch_build_emit(const int32_t* targets, int64_t T, int32_t V, int32_t P,
                               const uint32_t* bitmap, const int32_t* prefix,
-                              const int32_t* dev_status, int32_t* candidates,
+                              int32_t* dev_status, int32_t* candidates,
                               int32_t* target_pos, int32_t* vocab_pos, cudaStream_t s) {
   const int64_t n = (int64_t)V + T;
   const int blocks = (int)min64((n + 255) / 256, (int64_t)num_sms() * 8);

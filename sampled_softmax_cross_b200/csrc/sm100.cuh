@@ -394,6 +394,24 @@ constexpr uint32_t idesc_e4m3(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
+// ---------------------------------------------------------- bounds checks --
+// The bounds-checked build (compiled with SS_BOUNDS_CHECK=1 into
+// libsampled_ce_bounds.so) checks internal indices the kernels compute before
+// the access they guard: a failed check records SS_ERR_BAD_INDEX with detail
+// 200 + site in status[0..1] (first error wins) and the access is skipped. No
+// trap, no assert: the context stays usable. It stands in for a memory checker
+// where none can run. In the product build SS_CHECK is `true` and compiles away.
+#if defined(SS_BOUNDS_CHECK) && SS_BOUNDS_CHECK
+SS_DEV bool ss_check(bool ok, int32_t* status, int site) {
+  if (!ok && status != nullptr && atomicCAS(status, 0, 11 /* SS_ERR_BAD_INDEX */) == 0)
+    status[1] = 200 + site;
+  return ok;
+}
+#define SS_CHECK(cond, status, site) ::ssb::ss_check((cond), (status), (site))
+#else
+#define SS_CHECK(cond, status, site) true
+#endif
+
 // ------------------------------------------------------------------ misc --
 
 SS_DEV float ex2_approx(float x) {  // hardware 2^x (MUFU)

@@ -303,6 +303,7 @@ static ss_status forward_impl(const ss_bf16* x, const ss_bf16* lm_head,
   ra.partials = reinterpret_cast<double2*>(ws + L.partials);
   ra.loss = loss;
   ra.n_valid = n_valid;
+  ra.status = kstatus;
   uint8_t* x8 = ws + L.x8;
   uint8_t* w8 = ws + L.w8;
   float* qscale = reinterpret_cast<float*>(ws + L.qscale);

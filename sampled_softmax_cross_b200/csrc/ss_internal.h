@@ -17,7 +17,7 @@ cudaError_t launch_build_mark(const int32_t* targets, int64_t T, int32_t V, int3
                               int32_t* dev_status, cudaStream_t s);
 cudaError_t launch_build_emit(const int32_t* targets, int64_t T, int32_t V, int32_t P,
                               const uint32_t* bitmap, const int32_t* prefix,
-                              const int32_t* dev_status, int32_t* candidates,
+                              int32_t* dev_status, int32_t* candidates,
                               int32_t* target_pos, int32_t* vocab_pos, cudaStream_t s);
 cudaError_t launch_gather(const uint16_t* lm_head, const int32_t* cand, int32_t P, int32_t d,
                           int32_t V, uint16_t* w_c, int32_t* status, int32_t* zero_words,
@@ -49,6 +49,7 @@ struct RowArgs {
   const float* qscale;  // [3]: scale of x, of W_C, their product
   float* loss;          // [1] mean loss over valid rows
   int32_t* n_valid;     // [1]
+  int32_t* status;      // dev_status + 8 (kernel error, detail)
 };
 // Most blocks the row pass launches (the size of RowArgs::partials).
 constexpr int kRowPartials = 4096;

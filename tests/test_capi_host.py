@@ -162,3 +162,13 @@ def test_e4m3_host_rejections(lib):
     assert q(a, 12, a, a, a, None) == capi.STATUS["SS_ERR_INVALID_ARG"]  # n % 8
     assert q(a, 16, a, None, a, None) == capi.STATUS["SS_ERR_INVALID_ARG"]
     assert q(ctypes.c_void_p((1 << 20) + 8), 16, a, a, a, None) == capi.STATUS["SS_ERR_MISALIGNED"]
+
+
+def test_bounds_checked_build_exports_the_same_symbols():
+    """The bounds-checked variant (SS_BOUNDS_CHECK=1) builds from the same
+    sources and exports every declared entry point."""
+    path = build_lib.build(bounds_check=True)
+    assert path.endswith("libsampled_ce_bounds.so") and os.path.exists(path)
+    blib = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(blib, n), n
