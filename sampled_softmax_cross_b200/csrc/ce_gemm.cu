@@ -51,6 +51,7 @@
 //               swizzled shared-memory boxes and TMA stores; dX, dW: 16-byte stores)
 #include "sm100.cuh"
 #include "ce_gemm.h"
+#include "ss_internal.h"
 #include "sampled_ce.h"
 
 namespace ssb {
@@ -159,6 +160,8 @@ SS_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, 
 // [0] error, [1] detail (100 + 7), [2] 1 if warp 1 left through the flag,
 // [3] warp 0's wait in milliseconds.
 __global__ void __launch_bounds__(64, 1) k_wait_selftest(int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ __align__(8) uint64_t bars[2];
   __shared__ int abort_word;
   volatile int* abort_flag = &abort_word;
@@ -184,8 +187,7 @@ __global__ void __launch_bounds__(64, 1) k_wait_selftest(int32_t* status) {
 }
 
 cudaError_t launch_wait_selftest(int32_t* status, cudaStream_t s) {
-  k_wait_selftest<<<1, 64, 0, s>>>(status);
-  return cudaGetLastError();
+  return launch_pdl(k_wait_selftest, dim3(1), dim3(64), 0, s, status);
 }
 
 template <int KIND>
@@ -228,6 +230,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == 0 && lane == 0) {  // descriptors live in kernel parameter space
+    tma_prefetch_desc(&tma_a);
+    tma_prefetch_desc(&tma_b);
+  }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, TMEM_COLS);
     tmem_relinquish_pair();
@@ -236,13 +242,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
   cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // set-up above overlaps the previous kernel's tail; global memory only from here
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
-    if (lane == 0) {
-      tma_prefetch_desc(&tma_a);
-      tma_prefetch_desc(&tma_b);
-    }
     // B (W_C, or x' in dW) is reused by every tile: keep it in L2
     const uint64_t keep_b = policy_evict_last();
     int stage = 0;
@@ -647,12 +652,12 @@ cudaError_t launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b, co
                         const GemmArgs& args, int pairs, cudaStream_t s) {
   dim3 g(2 * pairs), blk(gemm_threads(kind));
   switch (kind) {
-    case KIND_FWD: k_gemm<KIND_FWD><<<g, blk, smem_bytes<KIND_FWD>(), s>>>(a, b, c, args); break;
-    case KIND_FWD8: k_gemm<KIND_FWD8><<<g, blk, smem_bytes<KIND_FWD8>(), s>>>(a, b, c, args); break;
-    case KIND_DX: k_gemm<KIND_DX><<<g, blk, smem_bytes<KIND_DX>(), s>>>(a, b, c, args); break;
-    default: k_gemm<KIND_DW><<<g, blk, smem_bytes<KIND_DW>(), s>>>(a, b, c, args); break;
+    case KIND_FWD: return launch_pdl(k_gemm<KIND_FWD>, g, blk, smem_bytes<KIND_FWD>(), s, a, b, c, args);
+    case KIND_FWD8:
+      return launch_pdl(k_gemm<KIND_FWD8>, g, blk, smem_bytes<KIND_FWD8>(), s, a, b, c, args);
+    case KIND_DX: return launch_pdl(k_gemm<KIND_DX>, g, blk, smem_bytes<KIND_DX>(), s, a, b, c, args);
+    default: return launch_pdl(k_gemm<KIND_DW>, g, blk, smem_bytes<KIND_DW>(), s, a, b, c, args);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace ssb

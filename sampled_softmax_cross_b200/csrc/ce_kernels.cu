@@ -78,6 +78,8 @@ __global__ void __cluster_dims__(kBuildCluster, 1, 1) __launch_bounds__(kBuildTh
     k_build_mark(const int32_t* __restrict__ targets, int64_t T, int32_t V, int32_t P,
                  int64_t offset, int32_t stride, uint32_t* __restrict__ g_bitmap,
                  int32_t* __restrict__ g_prefix, int32_t* __restrict__ st) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   extern __shared__ uint32_t bm[];
   __shared__ int s_warp[32];
   __shared__ int s_bad;
@@ -252,6 +254,8 @@ __global__ void k_build_emit(const int32_t* __restrict__ targets, int64_t T, int
                              const uint32_t* __restrict__ bitmap, const int32_t* __restrict__ prefix,
                              int32_t* __restrict__ st, int32_t* __restrict__ candidates,
                              int32_t* __restrict__ target_pos, int32_t* __restrict__ vocab_pos) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   const int code = *reinterpret_cast<const volatile int32_t*>(st);
   const int64_t n = (int64_t)V + T;
   for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n;
@@ -297,6 +301,8 @@ __global__ void k_gather(const uint4* __restrict__ lm, const int32_t* __restrict
                          int32_t vec_per_row, int32_t V, uint4* __restrict__ w_c,
                          int32_t* __restrict__ status, int32_t* __restrict__ zero_words,
                          int32_t n_zero_words) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < n_zero_words; i += blockDim.x) zero_words[i] = 0;
@@ -345,6 +351,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 __global__ void k_ref_logits(const uint4* __restrict__ x, const uint4* __restrict__ w_c,
                              const int32_t* __restrict__ tpos, int64_t T, int32_t vpr, int32_t P,
                              float* __restrict__ ref) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t pairs = (T + 1) / 2;  // two rows per warp iteration, all loads in flight
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -408,6 +416,8 @@ __device__ __forceinline__ int e4m3_scale_exp(float amax) {
 // the magnitude for finite values), by atomicMax.
 __global__ void k_amax_bf16(const uint4* __restrict__ a, int64_t na, const uint4* __restrict__ b,
                             int64_t nb, uint32_t* __restrict__ amax) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   uint32_t ma = 0, mb = 0;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   constexpr int U = 4;  // independent loads in flight per thread
@@ -453,6 +463,8 @@ __global__ void k_amax_bf16(const uint4* __restrict__ a, int64_t na, const uint4
 __global__ void k_quant_e4m3(const uint4* __restrict__ a, int64_t na, uint2* __restrict__ a8,
                              const uint4* __restrict__ b, int64_t nb, uint2* __restrict__ b8,
                              const uint32_t* __restrict__ amax, float* __restrict__ qscale) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   const int ka = e4m3_scale_exp(__uint_as_float(amax[0] << 16));
   const int kb = e4m3_scale_exp(__uint_as_float(amax[1] << 16));
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -499,6 +511,8 @@ __global__ void k_ref_logits_e4m3(const uint4* __restrict__ x8, const uint4* __r
                                   const int32_t* __restrict__ tpos, int64_t T, int32_t vpr,
                                   int32_t P, const float* __restrict__ qscale,
                                   float* __restrict__ ref) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const float s = __ldg(qscale + 2);
@@ -556,6 +570,8 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 a, float r) {
 constexpr int kRowsPerWarp = 8;
 
 __global__ void __launch_bounds__(256, 3) k_rows(RowArgs a) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   __shared__ double2 s_part[8];
   const int lane = threadIdx.x & 31;
   const int vpr = a.d / 8;
@@ -705,6 +721,8 @@ __device__ __forceinline__ float row_logit_any(const RowArgs& a, int64_t r, int6
 }
 
 __global__ void __launch_bounds__(kFinThreads) k_finalize(RowArgs a, int32_t nparts) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   __shared__ float sh[33];
   __shared__ float s_zt;
   __shared__ double s_sum[32], s_cnt[32];
@@ -801,6 +819,8 @@ __global__ void __launch_bounds__(kFinThreads) k_finalize(RowArgs a, int32_t npa
 // dW rows outside C (or every row) set to +0.0.
 __global__ void k_zero_rows(uint4* __restrict__ dW, int32_t V, int32_t vec_per_row,
                             const int32_t* __restrict__ vocab_pos, int all_rows) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < V; r += warps) {
@@ -821,6 +841,8 @@ __global__ void k_prefix_pos(const int32_t* __restrict__ prefix_table,
                              const int32_t* __restrict__ targets,
                              const int32_t* __restrict__ vocab_pos, int64_t T, int32_t V,
                              int32_t* __restrict__ prefix_pos, int32_t* __restrict__ status) {
+  pdl_wait();  // the previous kernel on the stream has completed
+  pdl_trigger();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < T; i += stride) {
     const int t = __ldg(targets + i);
@@ -874,9 +896,8 @@ cudaError_t launch_build_mark(const int32_t* targets, int64_t T, int32_t V, int3
     if (e != cudaSuccess) return e;
     g_build_attr[dev] = true;
   }
-  k_build_mark<<<kBuildCluster, kBuildThreads, smem, s>>>(targets, T, V, P, offset, stride,
+  return launch_pdl(k_build_mark, dim3(kBuildCluster), dim3(kBuildThreads), smem, s, targets, T, V, P, offset, stride,
                                                           bitmap, prefix, dev_status);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_build_emit(const int32_t* targets, int64_t T, int32_t V, int32_t P,
@@ -885,9 +906,8 @@ cudaError_t launch_build_emit(const int32_t* targets, int64_t T, int32_t V, int3
                               int32_t* target_pos, int32_t* vocab_pos, cudaStream_t s) {
   const int64_t n = (int64_t)V + T;
   const int blocks = (int)min64((n + 255) / 256, (int64_t)num_sms() * 8);
-  k_build_emit<<<blocks, 256, 0, s>>>(targets, T, V, P, bitmap, prefix, dev_status, candidates,
+  return launch_pdl(k_build_emit, dim3(blocks), dim3(256), 0, s, targets, T, V, P, bitmap, prefix, dev_status, candidates,
                                       target_pos, vocab_pos);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_gather(const uint16_t* lm_head, const int32_t* cand, int32_t P, int32_t d,
@@ -896,19 +916,17 @@ cudaError_t launch_gather(const uint16_t* lm_head, const int32_t* cand, int32_t 
   const int warps_per_block = 8;
   const int blocks = (int)min64((P + warps_per_block - 1) / warps_per_block,
                                        (int64_t)num_sms() * 16);
-  k_gather<<<blocks, warps_per_block * 32, 0, s>>>(reinterpret_cast<const uint4*>(lm_head), cand, P,
+  return launch_pdl(k_gather, dim3(blocks), dim3(warps_per_block * 32), 0, s, reinterpret_cast<const uint4*>(lm_head), cand, P,
                                                     d / 8, V, reinterpret_cast<uint4*>(w_c), status,
                                                     zero_words, n_zero_words);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_ref_logits(const uint16_t* x, const uint16_t* w_c, const int32_t* tpos,
                               int64_t T, int32_t d, int32_t P, float* ref, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int blocks = (int)min64(((T + 1) / 2 + 7) / 8, (int64_t)num_sms() * 16);
-  k_ref_logits<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(x),
+  return launch_pdl(k_ref_logits, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const uint4*>(x),
                                       reinterpret_cast<const uint4*>(w_c), tpos, T, d / 8, P, ref);
-  return cudaGetLastError();
 }
 
 static int rows_blocks(int64_t T) {
@@ -920,13 +938,11 @@ static int rows_blocks(int64_t T) {
 cudaError_t launch_rows(const RowArgs& a, cudaStream_t s) {
   const int blocks = rows_blocks(a.T);
   if (blocks == 0) return cudaSuccess;
-  k_rows<<<blocks, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k_rows, dim3(blocks), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_finalize(const RowArgs& a, cudaStream_t s) {
-  k_finalize<<<1, kFinThreads, 0, s>>>(a, rows_blocks(a.T));
-  return cudaGetLastError();
+  return launch_pdl(k_finalize, dim3(1), dim3(kFinThreads), 0, s, a, rows_blocks(a.T));
 }
 
 cudaError_t launch_prefix_pos(const int32_t* prefix_table, const int32_t* targets,
@@ -934,8 +950,7 @@ cudaError_t launch_prefix_pos(const int32_t* prefix_table, const int32_t* target
                               int32_t* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int blocks = (int)min64((T + 255) / 256, (int64_t)num_sms() * 8);
-  k_prefix_pos<<<blocks, 256, 0, s>>>(prefix_table, targets, vocab_pos, T, V, prefix_pos, status);
-  return cudaGetLastError();
+  return launch_pdl(k_prefix_pos, dim3(blocks), dim3(256), 0, s, prefix_table, targets, vocab_pos, T, V, prefix_pos, status);
 }
 
 cudaError_t launch_amax_bf16(const uint16_t* a, int64_t n, const uint16_t* b, int64_t m,
@@ -943,9 +958,8 @@ cudaError_t launch_amax_bf16(const uint16_t* a, int64_t n, const uint16_t* b, in
   const int64_t vec = (n + m) / 8;
   if (vec == 0) return cudaSuccess;
   const int blocks = (int)min64((vec + 255) / 256, (int64_t)num_sms() * 8);
-  k_amax_bf16<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(a), n / 8,
+  return launch_pdl(k_amax_bf16, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const uint4*>(a), n / 8,
                                      reinterpret_cast<const uint4*>(b), m / 8, amax);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_quant_e4m3(const uint16_t* a, int64_t n, uint8_t* a8, const uint16_t* b,
@@ -953,11 +967,10 @@ cudaError_t launch_quant_e4m3(const uint16_t* a, int64_t n, uint8_t* a8, const u
                               cudaStream_t s) {
   const int64_t vec = (n + m) / 8;
   const int blocks = (int)max64(1, min64((vec + 255) / 256, (int64_t)num_sms() * 8));
-  k_quant_e4m3<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(a), n / 8,
+  return launch_pdl(k_quant_e4m3, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const uint4*>(a), n / 8,
                                       reinterpret_cast<uint2*>(a8),
                                       reinterpret_cast<const uint4*>(b), m / 8,
                                       reinterpret_cast<uint2*>(b8), amax, qscale);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_ref_logits_e4m3(const uint8_t* x8, const uint8_t* w8, const int32_t* tpos,
@@ -965,17 +978,15 @@ cudaError_t launch_ref_logits_e4m3(const uint8_t* x8, const uint8_t* w8, const i
                                    float* ref, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int blocks = (int)min64((T + 7) / 8, (int64_t)num_sms() * 16);
-  k_ref_logits_e4m3<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(x8),
+  return launch_pdl(k_ref_logits_e4m3, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const uint4*>(x8),
                                            reinterpret_cast<const uint4*>(w8), tpos, T, d / 16, P,
                                            qscale, ref);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_zero_rows(uint16_t* dW, int32_t V, int32_t d, const int32_t* vocab_pos,
                              int all_rows, cudaStream_t s) {
   const int blocks = (int)min64((V + 7) / 8, (int64_t)num_sms() * 16);
-  k_zero_rows<<<blocks, 256, 0, s>>>(reinterpret_cast<uint4*>(dW), V, d / 8, vocab_pos, all_rows);
-  return cudaGetLastError();
+  return launch_pdl(k_zero_rows, dim3(blocks), dim3(256), 0, s, reinterpret_cast<uint4*>(dW), V, d / 8, vocab_pos, all_rows);
 }
 
 }  // namespace ssb

@@ -394,6 +394,17 @@ constexpr uint32_t idesc_e4m3(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
+// ------------------------------------------------ programmatic dependent launch --
+// Every kernel of the library is launched so that it may begin while the
+// previous kernel on the stream finishes (launch_pdl). Before its first access
+// to global memory a kernel waits until the previous grid has completed and
+// its writes are visible (griddepcontrol.wait; immediate when there is no such
+// grid); then it lets the next kernel begin launching (launch_dependents),
+// whose own wait again covers all of this grid. Work before the wait may only
+// touch shared memory, TMEM and kernel parameters.
+SS_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+SS_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------- bounds checks --
 // The bounds-checked build (compiled with SS_BOUNDS_CHECK=1 into
 // libsampled_ce_bounds.so) checks internal indices the kernels compute before

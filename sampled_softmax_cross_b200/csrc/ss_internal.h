@@ -11,6 +11,26 @@
 
 namespace ssb {
 
+// Launches `kernel` on `s` with programmatic stream serialization: the grid may
+// begin while the previous kernel on the stream is finishing. Every kernel of
+// the library waits (griddepcontrol.wait) before its first global-memory
+// access, so results are those of plain stream order.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Small kernels (ce_kernels.cu). Each returns the launch error.
 cudaError_t launch_build_mark(const int32_t* targets, int64_t T, int32_t V, int32_t P,
                               int64_t offset, int32_t stride, uint32_t* bitmap, int32_t* prefix,
