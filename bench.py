@@ -53,6 +53,9 @@ def parse():
                          "the gradient GEMMs stay bf16)")
     ap.add_argument("--no-dp-allreduce", action="store_true",
                     help="with N > 1: leave out the NCCL all-reduce of dW after each step")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a 256 MB buffer before every step, outside that step's events "
+                         "(each step then starts with a cold L2); value = tokens / sum of steps")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256,
@@ -306,6 +309,11 @@ def workload_config(w, n, dp=False):
             "l2": "no explicit flush: each step streams >2 GB of bf16 logits through HBM (L2 126 MB)"}
 
 
+def l2_note(args):
+    return ("flushed before every step: a 256 MB buffer written outside the step's events; value "
+            "= tokens / sum of the per-step times") if args.flush_l2 else None
+
+
 # ------------------------------------------------------------------ ours --
 
 def source_hash(*names):
@@ -490,11 +498,16 @@ def run_ours(args, w):
     capi.ss_timing_reset()
     capi.ss_timing_enable(True, gemms_only=True)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] if flush is not None else None
     clocks.start()
     barrier()
     torch.cuda.synchronize(dev)
     evs[0].record(stream)
     for k in range(args.steps):
+        if flush is not None:  # evict L2 (126 MB), then start this step's clock
+            flush.zero_()
+            starts[k].record(stream)
         step(k, timed_ar=True)
         evs[k + 1].record(stream)
     drain()
@@ -502,8 +515,12 @@ def run_ours(args, w):
     ev_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    ms = evs[0].elapsed_time(ev_end)
-    step_ms = [evs[k].elapsed_time(evs[k + 1]) for k in range(args.steps)]
+    if flush is None:
+        ms = evs[0].elapsed_time(ev_end)
+        step_ms = [evs[k].elapsed_time(evs[k + 1]) for k in range(args.steps)]
+    else:
+        step_ms = [starts[k].elapsed_time(evs[k + 1]) for k in range(args.steps)]
+        ms = float(sum(step_ms))
     ar_ms = [a.elapsed_time(b) for a, b in ar_ev]
     clk = clocks.stop()
     capi.ss_timing_enable(False)
@@ -630,7 +647,7 @@ def run_ours(args, w):
             "dtype": "bf16" if args.precision == "bf16" else "e4m3 logits GEMM, bf16 gradient GEMMs",
             "precision": args.precision,
             "data": "synthetic (seeded Zipf targets, N(0,1) x, N(0,1/d) lm_head)",
-            "config": workload_config(w, world, dp),
+            "config": dict(workload_config(w, world, dp), **({"l2": l2_note(args)} if args.flush_l2 else {})),
             "step_tflops": step_tflops,
             "frac_of_bf16_peak": {"burst": step_tflops / pk["bf16"],
                                   "sustained": step_tflops / pk["bf16_sus"],

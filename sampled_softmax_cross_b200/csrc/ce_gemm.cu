@@ -46,9 +46,10 @@
 //               the e4m3 forward, 4 x 48 KB in dX and dW
 //   warp 1      TMEM owner (2 x 256 columns); in the leader, the MMA issuer
 //               (kind::f16, or kind::f8f6f4 with K=32 for the e4m3 forward)
-//   warps 2..   epilogue, 4 warps (8 in the e4m3 forward, two per TMEM lane
-//               quarter): TMEM -> registers -> math -> global (forward: through
-//               swizzled shared-memory boxes and TMA stores; dX, dW: 16-byte stores)
+//   warps 2..   epilogue: 8 warps in the forwards (two per TMEM lane quarter,
+//               each over half of a tile's columns), 4 in dX and dW:
+//               TMEM -> registers -> math -> global (forward: through swizzled
+//               shared-memory boxes and TMA stores; dX, dW: 16-byte stores)
 #include "sm100.cuh"
 #include "ce_gemm.h"
 #include "ss_internal.h"
@@ -70,20 +71,21 @@ constexpr float LOG2E = 1.4426950408889634f;
 // Per kind: operand majors, the E store path, pipeline stages and epilogue
 // warps. The forward stores the 2.4 GB E stream through staging boxes and
 // TMA bulk stores (1.47 ms against 1.89 ms with 16-byte register stores,
-// measured); the boxes cost one operand stage. With e4m3 operands the MMAs
-// of a tile take half as long (6 K blocks of 128 at twice the rate), and the
-// epilogue -- TMEM loads, an exponential per element, packing, staging and
-// stores -- becomes the longer part: that kind gets two warps per TMEM lane
-// quarter, each taking half of the tile's columns (8% faster measured; the
-// bf16 forward gains nothing from it). dX and dW (hundreds of K blocks per
+// measured); the boxes cost one operand stage. Its epilogue -- TMEM loads, an
+// exponential per element, packing, staging and stores -- is busy for most of
+// the kernel, stalled on dependency latency with one warp per scheduler: both
+// forwards run two warps per TMEM lane quarter, each over half of the tile's
+// columns (bf16: 3% faster with one staging box per warp, measured; two boxes
+// per warp and one stage fewer gained nothing; e4m3, whose MMAs take half as
+// long: 8% faster). dX and dW (hundreds of K blocks per
 // tile) store little, from registers; their 48 KB stages (two A blocks) fit
 // four times, 192 KB in flight per SM as with seven 32 KB stages.
 template <int KIND>
 struct Op;
 template <>
 struct Op<KIND_FWD> {  // A = x (K-major), B = W_C (K-major)
-  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6, EPI_WARPS = 4, AB = 1,
-                       EPI_BUFS = 2;
+  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6, EPI_WARPS = 8, AB = 1,
+                       EPI_BUFS = 1;
 };
 template <>
 struct Op<KIND_FWD8> {  // A = x_q, B = W_C,q (e4m3, K-major; 128 per K block)

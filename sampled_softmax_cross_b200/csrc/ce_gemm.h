@@ -9,9 +9,9 @@
 namespace ssb {
 
 // Partial row sums the forward epilogue writes per 256-column tile: one per
-// epilogue warp sharing a TMEM lane quarter (the e4m3 forward has two, each
-// over half of the tile's columns).
-constexpr int kFwdSumsPerTileBf16 = 1, kFwdSumsPerTileE4m3 = 2;
+// epilogue warp sharing a TMEM lane quarter (two, each over half of the
+// tile's columns).
+constexpr int kFwdSumsPerTileBf16 = 2, kFwdSumsPerTileE4m3 = 2;
 
 // Arguments of the three tcgen05 GEMMs (forward logits, dX, dW_C).
 struct GemmArgs {
