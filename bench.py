@@ -643,6 +643,7 @@ def run_ours(args, w):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
             "ms_per_step_median": med_max,
+            "step_ms": [round(x, 4) for x in step_ms],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if args.precision == "bf16" else "e4m3 logits GEMM, bf16 gradient GEMMs",
             "precision": args.precision,

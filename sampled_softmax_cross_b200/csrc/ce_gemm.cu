@@ -80,27 +80,40 @@ constexpr float LOG2E = 1.4426950408889634f;
 // long: 8% faster). dX and dW (hundreds of K blocks per
 // tile) store little, from registers; their 48 KB stages (two A blocks) fit
 // four times, 192 KB in flight per SM as with seven 32 KB stages.
+// What the kernel computes: the forward (logits and E), dX, or dW_C with its scatter.
+enum Role { ROLE_FWD = 0, ROLE_DX = 1, ROLE_DW = 2 };
+
 template <int KIND>
 struct Op;
 template <>
 struct Op<KIND_FWD> {  // A = x (K-major), B = W_C (K-major)
-  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6, EPI_WARPS = 8, AB = 1,
-                       EPI_BUFS = 1;
+  static constexpr int ROLE = ROLE_FWD, A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 6,
+                       EPI_WARPS = 8, AB = 1, EPI_BUFS = 1;
 };
 template <>
 struct Op<KIND_FWD8> {  // A = x_q, B = W_C,q (e4m3, K-major; 128 per K block)
-  static constexpr int A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 5, EPI_WARPS = 8, AB = 1,
-                       EPI_BUFS = 2;
+  static constexpr int ROLE = ROLE_FWD, A_MN = 0, B_MN = 0, TMA_STORE = 1, STAGES = 5,
+                       EPI_WARPS = 8, AB = 1, EPI_BUFS = 2;
 };
 template <>
 struct Op<KIND_DX> {  // A = E' (K-major), B = W_C viewed [K=P][N=d] (MN-major)
-  static constexpr int A_MN = 0, B_MN = 1, TMA_STORE = 0, STAGES = 4, EPI_WARPS = 4, AB = 2,
-                       EPI_BUFS = 0;
+  static constexpr int ROLE = ROLE_DX, A_MN = 0, B_MN = 1, TMA_STORE = 0, STAGES = 4,
+                       EPI_WARPS = 4, AB = 2, EPI_BUFS = 0;
 };
 template <>
 struct Op<KIND_DW> {  // A = E' viewed [K=T][M=P] (MN-major), B = x' viewed [K=T][N=d] (MN-major)
-  static constexpr int A_MN = 1, B_MN = 1, TMA_STORE = 0, STAGES = 4, EPI_WARPS = 4, AB = 2,
-                       EPI_BUFS = 0;
+  static constexpr int ROLE = ROLE_DW, A_MN = 1, B_MN = 1, TMA_STORE = 0, STAGES = 4,
+                       EPI_WARPS = 4, AB = 2, EPI_BUFS = 0;
+};
+template <>
+struct Op<KIND_DX1> {  // dX on 256-row tiles: 7 stages of 32 KB, two accumulators
+  static constexpr int ROLE = ROLE_DX, A_MN = 0, B_MN = 1, TMA_STORE = 0, STAGES = 7,
+                       EPI_WARPS = 4, AB = 1, EPI_BUFS = 0;
+};
+template <>
+struct Op<KIND_DW1> {  // dW on 256-row tiles
+  static constexpr int ROLE = ROLE_DW, A_MN = 1, B_MN = 1, TMA_STORE = 0, STAGES = 7,
+                       EPI_WARPS = 4, AB = 1, EPI_BUFS = 0;
 };
 
 // Bytes of one pipeline stage: AB blocks of 128 A rows, and the CTA's half of B.
@@ -133,8 +146,8 @@ constexpr int smem_bytes() {
   return 1024 + Op<KIND>::STAGES * stage_bytes<KIND>() + epi_bytes<KIND>() + BAR_BYTES;
 }
 static_assert(smem_bytes<KIND_FWD>() <= 232448 && smem_bytes<KIND_FWD8>() <= 232448 &&
-                  smem_bytes<KIND_DX>() <= 232448 &&
-                  smem_bytes<KIND_DW>() <= 232448,
+                  smem_bytes<KIND_DX>() <= 232448 && smem_bytes<KIND_DW>() <= 232448 &&
+                  smem_bytes<KIND_DX1>() <= 232448 && smem_bytes<KIND_DW1>() <= 232448,
               "shared memory budget");
 
 SS_DEV void raise_abort(volatile int* abort_flag, int32_t* status, int kind) {
@@ -381,7 +394,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
       const int nv = __ldg(args.n_valid);
       scale = nv > 0 ? __ldg(args.grad_loss) / (float)nv : 0.f;
     }
-    if (KIND == KIND_DW && args.vocab_pos != nullptr) {
+    if (Op<KIND>::ROLE == ROLE_DW && args.vocab_pos != nullptr) {
       // The rows of dW outside C are +0.0. The epilogue warps of every CTA
       // write them while the first tiles' MMAs run (they are disjoint from
       // the rows the tiles scatter). Each warp takes blocks of 32 classes.
@@ -424,11 +437,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
         ref2_1 = __ldg(args.ref + row0 + 2 * BM) * LOG2E;
         keep1 = __ldg(args.tpos + row0 + 2 * BM) >= 0;
       }
-      if (KIND == KIND_DX) {
+      if (Op<KIND>::ROLE == ROLE_DX) {
         rs0 = row0 < args.M ? scale * __ldg(args.rscale + row0) : 0.f;
         if (AB > 1) rs1 = row0 + 2 * BM < args.M ? scale * __ldg(args.rscale + row0 + 2 * BM) : 0.f;
       }
-      if (KIND == KIND_DW) {
+      if (Op<KIND>::ROLE == ROLE_DW) {
         if (row0 < args.M) cls0 = __ldg(args.cand + row0);
         if (AB > 1 && row0 + 2 * BM < args.M) cls1 = __ldg(args.cand + row0 + 2 * BM);
       }
@@ -499,7 +512,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
 #pragma unroll
               for (int j = 0; j < 64; ++j) v[j] = 0.f;
             }
-          } else if (KIND == KIND_DX) {
+          } else if (Op<KIND>::ROLE == ROLE_DX) {
 #pragma unroll
             for (int j = 0; j < 64; ++j) v[j] *= rs;
           } else {
@@ -533,7 +546,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
               bulk_commit();
             }
             ++store_ctr;
-          } else if (KIND != KIND_DW) {
+          } else if (Op<KIND>::ROLE != ROLE_DW) {
             // bf16 row segment straight from registers (16-byte stores)
             if (row_ok) {
               uint4* dst = reinterpret_cast<uint4*>(args.out + (size_t)row * args.ld_out + col0);
@@ -598,6 +611,8 @@ int gemm_tile_rows(int kind) {
     case KIND_FWD: return 2 * BM * Op<KIND_FWD>::AB;
     case KIND_FWD8: return 2 * BM * Op<KIND_FWD8>::AB;
     case KIND_DX: return 2 * BM * Op<KIND_DX>::AB;
+    case KIND_DX1: return 2 * BM * Op<KIND_DX1>::AB;
+    case KIND_DW1: return 2 * BM * Op<KIND_DW1>::AB;
     default: return 2 * BM * Op<KIND_DW>::AB;
   }
 }
@@ -607,6 +622,8 @@ int gemm_smem_bytes(int kind) {
     case KIND_FWD: return smem_bytes<KIND_FWD>();
     case KIND_FWD8: return smem_bytes<KIND_FWD8>();
     case KIND_DX: return smem_bytes<KIND_DX>();
+    case KIND_DX1: return smem_bytes<KIND_DX1>();
+    case KIND_DW1: return smem_bytes<KIND_DW1>();
     default: return smem_bytes<KIND_DW>();
   }
 }
@@ -616,6 +633,8 @@ const void* gemm_kernel_ptr(int kind) {
     case KIND_FWD: return reinterpret_cast<const void*>(&k_gemm<KIND_FWD>);
     case KIND_FWD8: return reinterpret_cast<const void*>(&k_gemm<KIND_FWD8>);
     case KIND_DX: return reinterpret_cast<const void*>(&k_gemm<KIND_DX>);
+    case KIND_DX1: return reinterpret_cast<const void*>(&k_gemm<KIND_DX1>);
+    case KIND_DW1: return reinterpret_cast<const void*>(&k_gemm<KIND_DW1>);
     default: return reinterpret_cast<const void*>(&k_gemm<KIND_DW>);
   }
 }
@@ -626,6 +645,8 @@ int gemm_threads(int kind) {
     case KIND_FWD: return num_threads<KIND_FWD>();
     case KIND_FWD8: return num_threads<KIND_FWD8>();
     case KIND_DX: return num_threads<KIND_DX>();
+    case KIND_DX1: return num_threads<KIND_DX1>();
+    case KIND_DW1: return num_threads<KIND_DW1>();
     default: return num_threads<KIND_DW>();
   }
 }
@@ -658,6 +679,10 @@ cudaError_t launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b, co
     case KIND_FWD8:
       return launch_pdl(k_gemm<KIND_FWD8>, g, blk, smem_bytes<KIND_FWD8>(), s, a, b, c, args);
     case KIND_DX: return launch_pdl(k_gemm<KIND_DX>, g, blk, smem_bytes<KIND_DX>(), s, a, b, c, args);
+    case KIND_DX1:
+      return launch_pdl(k_gemm<KIND_DX1>, g, blk, smem_bytes<KIND_DX1>(), s, a, b, c, args);
+    case KIND_DW1:
+      return launch_pdl(k_gemm<KIND_DW1>, g, blk, smem_bytes<KIND_DW1>(), s, a, b, c, args);
     default: return launch_pdl(k_gemm<KIND_DW>, g, blk, smem_bytes<KIND_DW>(), s, a, b, c, args);
   }
 }

@@ -40,8 +40,10 @@ struct GemmArgs {
 };
 
 // KIND_FWD8: the forward on e4m3 operands (x and W_C quantized per tensor).
-enum GemmKind { KIND_FWD = 0, KIND_DX = 1, KIND_DW = 2, KIND_FWD8 = 3 };
-constexpr int kNumGemmKinds = 4;
+// KIND_DX, KIND_DW: 512-row tiles; KIND_DX1, KIND_DW1: the same GEMMs on
+// 256-row tiles, for shapes where 512-row tiles would leave a poor last wave.
+enum GemmKind { KIND_FWD = 0, KIND_DX = 1, KIND_DW = 2, KIND_FWD8 = 3, KIND_DX1 = 4, KIND_DW1 = 5 };
+constexpr int kNumGemmKinds = 6;
 
 // Launches `pairs` CTA pairs (clusters of 2) of the persistent GEMM kernel.
 cudaError_t launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b,
