@@ -347,6 +347,19 @@ def test_full_size_workload_compared_in_full(name):
     compare_full(g, o, t)
 
 
+def test_ragged_512_row_backward_tiles_compared_in_full():
+    """T = 45000 and P = 20000 (d = 768): both backward GEMMs run on 512-row
+    tiles (4 and 2 waves of CTA pairs, against 8 and 4 with 256-row tiles), and
+    neither T nor P is a multiple of 512, so the last tile of each has rows
+    past the end (456 and 32 rows in it). Every output against the oracle."""
+    T, d, V, P = 45000, 768, 50304, 20000
+    x, lm, t = wl.make_inputs(T, d, V, 1.05, 0.01, 45)
+    assert np.unique(t[t >= 0]).size <= P
+    g = run_path(x, lm, t, P, 777)
+    o = oracle_run(x, lm, t, P, 777)
+    compare_full(g, o, t)
+
+
 @pytest.mark.parametrize("name,d", [("tiny", None), ("stage0", None), ("stage2_early", None),
                                     ("stage2_late", None), ("full_softmax", None),
                                     ("ragged_d", 200)])
