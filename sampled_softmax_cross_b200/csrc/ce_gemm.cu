@@ -128,6 +128,9 @@ constexpr int acc_bufs() {
   return Op<KIND>::AB == 1 ? 2 : 1;
 }
 
+static_assert(!Op<KIND_DX>::TMA_STORE && !Op<KIND_DW>::TMA_STORE && !Op<KIND_DX1>::TMA_STORE &&
+                  !Op<KIND_DW1>::TMA_STORE,
+              "only the forwards stage E for TMA stores");
 static_assert(Op<KIND_FWD>::EPI_WARPS / 4 == kFwdSumsPerTileBf16 &&
                   Op<KIND_FWD8>::EPI_WARPS / 4 == kFwdSumsPerTileE4m3,
               "row sums per tile");
@@ -149,6 +152,17 @@ static_assert(smem_bytes<KIND_FWD>() <= 232448 && smem_bytes<KIND_FWD8>() <= 232
                   smem_bytes<KIND_DX>() <= 232448 && smem_bytes<KIND_DW>() <= 232448 &&
                   smem_bytes<KIND_DX1>() <= 232448 && smem_bytes<KIND_DW1>() <= 232448,
               "shared memory budget");
+
+// One lane's 64 values of a chunk, as bf16, into row `lane` of a 32 x 64
+// staging box with the 128-byte swizzle of the E store's tensor map.
+SS_DEV void stage_box(uint32_t row_addr, int lane, const float (&v)[64]) {
+#pragma unroll
+  for (int cc = 0; cc < 8; ++cc) {
+    st_shared_v4(row_addr + ((cc ^ (lane & 7)) << 4), pack_bf16x2(v[cc * 8 + 0], v[cc * 8 + 1]),
+                 pack_bf16x2(v[cc * 8 + 2], v[cc * 8 + 3]), pack_bf16x2(v[cc * 8 + 4], v[cc * 8 + 5]),
+                 pack_bf16x2(v[cc * 8 + 6], v[cc * 8 + 7]));
+  }
+}
 
 SS_DEV void raise_abort(volatile int* abort_flag, int32_t* status, int kind) {
   *abort_flag = 1;
@@ -523,27 +537,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
           if (Op<KIND>::TMA_STORE) {
             // bf16 tile -> swizzled staging box -> TMA store
             constexpr int NB = Op<KIND>::EPI_BUFS > 0 ? Op<KIND>::EPI_BUFS : 1;
-            uint8_t* buf = epi_smem + (e * NB + (int)(store_ctr % NB)) * EPI_BUF;
-            if (lane == 0) bulk_wait_read<NB - 1>();  // this buffer's last store has read it
-            __syncwarp();
-            const uint32_t base = smem_u32(buf) + lane * 128;
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-              st_shared_v4(base + ((cc ^ (lane & 7)) << 4),
-                           pack_bf16x2(v[cc * 8 + 0], v[cc * 8 + 1]),
-                           pack_bf16x2(v[cc * 8 + 2], v[cc * 8 + 3]),
-                           pack_bf16x2(v[cc * 8 + 4], v[cc * 8 + 5]),
-                           pack_bf16x2(v[cc * 8 + 6], v[cc * 8 + 7]));
-            }
-            fence_async_smem();
-            __syncwarp();
-            const int box_row = row - lane;  // first row of this warp's 32-row box
-            if (lane == 0 && box_row < args.M) {
-              if (IS_FWD)
+            const uint32_t lane_off = lane * 128;
+            const int box_row = row - lane;  // first row of this warp's 32-row boxes
+            if (NB >= CPW) {
+              // a box per chunk of this warp's columns: one async-proxy fence and
+              // one bulk group for all of them (e4m3 forward: 2% faster, measured)
+              const int slot = c - c_begin;
+              uint8_t* buf = epi_smem + (e * NB + slot) * EPI_BUF;
+              if (slot == 0) {  // the previous tile's stores have read this warp's boxes
+                if (lane == 0) bulk_wait_read<0>();
+                __syncwarp();
+              }
+              stage_box(smem_u32(buf) + lane_off, lane, v);
+              if (c == c_end - 1) {
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0 && box_row < args.M) {
+                  for (int sl = 0; sl <= slot; ++sl)
+                    tma_store_2d_hint(&tma_c, epi_smem + (e * NB + sl) * EPI_BUF,
+                                      n0 + (c_begin + sl) * 64, box_row, store_policy);
+                  bulk_commit();
+                }
+              }
+            } else {
+              // a ring of NB boxes: fence and store each chunk as it is staged
+              uint8_t* buf = epi_smem + (e * NB + (int)(store_ctr % NB)) * EPI_BUF;
+              if (lane == 0) bulk_wait_read<NB - 1>();  // this buffer's last store has read it
+              __syncwarp();
+              stage_box(smem_u32(buf) + lane_off, lane, v);
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0 && box_row < args.M) {
                 tma_store_2d_hint(&tma_c, buf, col0, box_row, store_policy);
-              else
-                tma_store_2d(&tma_c, buf, col0, box_row);
-              bulk_commit();
+                bulk_commit();
+              }
             }
             ++store_ctr;
           } else if (Op<KIND>::ROLE != ROLE_DW) {
