@@ -139,6 +139,17 @@ def test_e4m3_headline_workload():
     check_grad(wl.bits_to_f64(g["dW_bits"][cand[cols]]), dw_o, "dW rows")
 
 
+def test_e4m3_stage0_compared_in_full():
+    """stage0 at full size (T=16384, d=768, P=10240) in e4m3: every output
+    against the oracle's e4m3 path -- codes, candidate set and positions bit
+    for bit, loss, lse, and every element of dX and dW."""
+    w = wl.WORKLOADS["stage0"]
+    x, lm, t = wl.workload_inputs(w)
+    g = run_path(x, lm, t, w.P, w.offset, precision="e4m3")
+    o = _e4m3_oracle(x, lm, t, w.P, w.offset)
+    compare_full(g, o, t)
+
+
 def test_e4m3_empty_microbatch_and_full_vocabulary():
     lm = wl.bf16_bits(np.random.default_rng(0).standard_normal((512, 64), dtype=np.float32))
     g = run_path(np.zeros((0, 64), np.uint16), lm, np.zeros(0, np.int32), 100, 4,
