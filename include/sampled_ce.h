@@ -18,7 +18,11 @@
  *     allocates no device memory and keeps no state between calls, apart
  *     from per-device launch attributes it sets once.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). All work
- *     is enqueued on it; no call synchronises the device.
+ *     is enqueued on it; no call synchronises the device. Kernels are
+ *     launched with programmatic stream serialization: each may begin while
+ *     the previous kernel on the stream finishes, and waits for it to complete
+ *     before touching global memory, so results are those of plain stream
+ *     order (a caller's own kernels launched normally are unaffected).
  *   - Host-detectable errors (sizes, alignment, workspace too small, a
  *     stride not coprime with V, a device that is not sm_100) return a
  *     non-zero ss_status before anything is enqueued. Errors that only the
@@ -264,11 +268,13 @@ SS_API ss_status ss_selftest_wait_limit(int32_t* dev_status, void* stream);
 
 /* Kernel timing for diagnostics. While enabled, each kernel launch the library
  * makes is bracketed by two CUDA events recorded on its stream (a pool of
- * 8192 launches; later launches go untimed); enable = 2 brackets only the
- * tensor-core GEMM launches (fewer events in a timed loop), 1 every launch,
- * 0 none. ss_timing_query synchronises on the recorded events and returns,
- * for the i-th distinct kernel name, its launch count and total
- * milliseconds. Not thread-safe; for benchmarks. */
+ * 8192 launches, created by the first enabling call so that none is created
+ * inside a timed region; later launches go untimed); enable = 2 brackets only
+ * the tensor-core GEMM launches (fewer events in a timed loop), 1 every
+ * launch, 0 none. An event between two launches also ends the overlap the
+ * programmatic launch allows there. ss_timing_query synchronises on the
+ * recorded events and returns, for the i-th distinct kernel name, its launch
+ * count and total milliseconds. Not thread-safe; for benchmarks. */
 SS_API ss_status ss_timing_enable(int32_t enable);
 SS_API ss_status ss_timing_reset(void);
 SS_API int32_t ss_timing_count(void);
