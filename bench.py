@@ -13,7 +13,10 @@ microbatch (seed + rank, negative-window offset staggered by V*rank/N): weak
 scaling, timed as the max over ranks. The path itself has no collective; the
 data-parallel gradient sync of the dense dW [V, d] (an NCCL all-reduce, on its
 own stream, overlapping the next step's build and forward) runs inside the
-timed region unless --no-dp-allreduce is given.
+timed region unless --no-dp-allreduce is given. Launched by
+torch.distributed.run with one process, the bench forms a one-rank NCCL group
+and runs the same gradient-sync code (the all-reduce of one rank is a no-op on
+the data, but the streams, events and double-buffered dW are all exercised).
 """
 
 from __future__ import annotations
@@ -52,7 +55,8 @@ def parse():
                     help="operands of the logits GEMM (e4m3: per-tensor scaled 8-bit floats; "
                          "the gradient GEMMs stay bf16)")
     ap.add_argument("--no-dp-allreduce", action="store_true",
-                    help="with N > 1: leave out the NCCL all-reduce of dW after each step")
+                    help="under torch.distributed.run: leave out the NCCL all-reduce of dW "
+                         "after each step")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 256 MB buffer before every step, outside that step's events "
                          "(each step then starts with a cold L2); value = tokens / sum of steps")
@@ -290,7 +294,8 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, args.gpus, args.gpus > 1 and not args.no_dp_allreduce),
+        "config": workload_config(w, args.gpus, launched_grouped(args.gpus)
+                                  and not args.no_dp_allreduce),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -304,7 +309,7 @@ def workload_config(w, n, dp=False):
             "T": w.T, "d": w.d, "V": w.V, "P": w.P, "offset": w.offset, "zipf_s": w.zipf_s,
             "ignored_frac": w.ignore_frac, "seed": w.seed,
             "parallelism": (f"dp{n} (independent microbatch per rank" +
-                            (", dW all-reduced over the ranks after each step)" if n > 1 and dp
+                            (", dW all-reduced over the ranks after each step)" if dp
                              else ", no collective)")),
             "l2": "no explicit flush: each step streams >2 GB of bf16 logits through HBM (L2 126 MB)"}
 
@@ -312,6 +317,12 @@ def workload_config(w, n, dp=False):
 def l2_note(args):
     return ("flushed before every step: a 256 MB buffer written outside the step's events; value "
             "= tokens / sum of the per-step times") if args.flush_l2 else None
+
+
+def launched_grouped(world):
+    """True where the bench runs in a process group: more than one rank, or one
+    rank that torch.distributed.run launched."""
+    return world > 1 or ("MASTER_ADDR" in os.environ and "RANK" in os.environ)
 
 
 # ------------------------------------------------------------------ ours --
@@ -402,7 +413,7 @@ def run_e2e(args, w, world, dev, x_bits, lm_bits, targets, offset, barrier, dist
     ev1.record(s_out)
     torch.cuda.synchronize(dev)
     barrier()
-    e_ms = ranks.max_over_ranks(ev0.elapsed_time(ev1), dist if world > 1 else None, dev)
+    e_ms = ranks.max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
     h2d = hx.numel() * 2 + hlm.numel() * 2 + ht.numel() * 4
     d2h = 4 + sets[0]["hdx"].numel() * 2 + sets[0]["hdW"].numel() * 2
     st = sets[1]["ce"].status()
@@ -423,18 +434,19 @@ def run_ours(args, w):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
+    grouped = launched_grouped(world)
+    if grouped:
         torch.cuda.set_device(local)
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", local if world > 1 else 0)
+    dev = torch.device("cuda", local if grouped else 0)
     torch.cuda.set_device(dev)
     if rank == 0:
         build_lib.build()
-    if world > 1:
+    if grouped:
         dist.barrier()
     capi.load()
-    dp = world > 1 and not args.no_dp_allreduce
+    dp = grouped and not args.no_dp_allreduce
 
     # this rank's microbatch: own seed, staggered window start
     x_bits, lm_bits, targets = wl.make_inputs(w.T, w.d, w.V, w.zipf_s, w.ignore_frac,
@@ -479,7 +491,7 @@ def run_ours(args, w):
                 stream.wait_event(e)
 
     def barrier():
-        if world > 1:
+        if grouped:
             dist.barrier()
 
     for k in range(args.warmup):
@@ -544,8 +556,8 @@ def run_ours(args, w):
     # launches of this library in the timed loop: the per-step count times the steps
     launches = sum(n for n, _ in every.values()) * args.steps // n_sep
 
-    ms_max = ranks.max_over_ranks(ms, dist if world > 1 else None, dev)
-    med_max = ranks.max_over_ranks(float(np.median(step_ms)), dist if world > 1 else None, dev)
+    ms_max = ranks.max_over_ranks(ms, dist, dev)
+    med_max = ranks.max_over_ranks(float(np.median(step_ms)), dist, dev)
 
     # e2e: the same step from pinned host buffers, copies inside the timed region
     e2e = None
@@ -677,7 +689,7 @@ def run_ours(args, w):
                         "on its own stream, overlapping the next step's build and forward",
                 "bytes": w.V * w.d * 2, "avg_ms": float(np.mean(ar_ms)) if ar_ms else None}
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if grouped:
         dist.barrier()
         dist.destroy_process_group()
 
