@@ -40,6 +40,13 @@
 //             SMs (about 11 TB/s measured) bounds these GEMMs, not the tensor
 //             cores. Their K loops are hundreds of blocks long, so a
 //             single-buffered accumulator costs under 1%.
+// Tiles go to CTA pairs dynamically: each pair starts on tile `cluster` and
+// then takes the next index from a counter in global memory (atomicAdd by the
+// leader's producer, which passes it to both CTAs' warps through a small ring
+// in shared memory), so pairs that start late -- their SMs still held by a
+// kernel on another stream, such as a gradient all-reduce -- take fewer
+// tiles instead of ending the kernel late. Tiles are taken in n-fastest
+// order, so the pairs running at once share the A stripe.
 // Per CTA, persistent over tiles:
 //   warp 0      TMA producer, ring of stages (A 128x64 per block + B 128x64
 //               bf16, or 128x128 e4m3 codes): 6 x 32 KB in the forward, 5 in
@@ -65,6 +72,16 @@ constexpr int A_STAGE = BM * BK * 2;   // 16 KB
 constexpr int B_STAGE = BNH * BK * 2;  // 16 KB
 constexpr int EPI_BUF = 32 * 64 * 2;  // one 32-row x 64-column bf16 box (4 KB)
 constexpr int BAR_BYTES = 256;
+// Slots of the tile-index ring. A slot is rewritten SCHED tiles after it was
+// written, and by then every warp of the pair has read it: when the leader's
+// producer starts tile s, the MMA warp has finished K block s * num_kb - 1 -
+// STAGES (the stage it reloads), so it works on tile >= s - ceil(STAGES /
+// num_kb) and the epilogue warps of both CTAs, which released that tile's
+// accumulator ACC tiles earlier, have read the slot of tile s - ceil(STAGES /
+// num_kb) - ACC - 1 or later; the peer's producer has loaded as far as the MMA
+// warp has computed. So SCHED >= ceil(STAGES / num_kb) + ACC + 1, at most
+// 7 + 2 + 1 here, is enough.
+constexpr int SCHED = 12;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -148,6 +165,16 @@ template <int KIND>
 constexpr int smem_bytes() {
   return 1024 + Op<KIND>::STAGES * stage_bytes<KIND>() + epi_bytes<KIND>() + BAR_BYTES;
 }
+// barriers (full, empty per stage; tfull, tempty), the ring's slots, the TMEM
+// address and the abort flag
+template <int KIND>
+constexpr int bar_bytes_used() {
+  return (2 * Op<KIND>::STAGES + 4 + SCHED) * 8 + 8;
+}
+static_assert(bar_bytes_used<KIND_FWD>() <= BAR_BYTES && bar_bytes_used<KIND_FWD8>() <= BAR_BYTES &&
+                  bar_bytes_used<KIND_DX>() <= BAR_BYTES && bar_bytes_used<KIND_DW>() <= BAR_BYTES &&
+                  bar_bytes_used<KIND_DX1>() <= BAR_BYTES && bar_bytes_used<KIND_DW1>() <= BAR_BYTES,
+              "barrier region");
 static_assert(smem_bytes<KIND_FWD>() <= 232448 && smem_bytes<KIND_FWD8>() <= 232448 &&
                   smem_bytes<KIND_DX>() <= 232448 && smem_bytes<KIND_DW>() <= 232448 &&
                   smem_bytes<KIND_DX1>() <= 232448 && smem_bytes<KIND_DW1>() <= 232448,
@@ -178,6 +205,53 @@ SS_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, 
   ok = __all_sync(0xffffffffu, ok);
   if (!ok) raise_abort(abort_flag, status, kind);
   return ok;
+}
+
+// The tile-index ring. Slot `it % SCHED` holds {it + 1, tile}: the tile that
+// follows a warp's `it`-th tile (an index >= the tile count ends the warp's
+// loop). The leader's producer writes both CTAs' copies with plain 64-bit
+// stores (the peer's through its shared::cluster address); the other warps
+// of the pair (the leader's MMA warp, the peer's producer, the epilogue warps
+// of both CTAs) poll their own copy until its tag is it + 1. The value is its
+// own flag, so neither side needs a fence or a barrier, and the slot is not
+// rewritten before every warp has read it (SCHED, above). A tag past it + 1
+// would mean a warp fell behind that bound: it is reported, not used.
+SS_DEV void ring_publish(volatile uint64_t* ring, int it, int tile) {
+  if ((threadIdx.x & 31) == 0) {
+    const int j = it % SCHED;
+    const uint64_t v = ((uint64_t)((uint32_t)it + 1u) << 32) | (uint32_t)tile;
+    ring[j] = v;
+    st_shared_cluster_u64(mapa_shared(smem_u32((const void*)(ring + j)), 1), v);
+  }
+  __syncwarp();
+}
+
+SS_DEV bool ring_next(const volatile uint64_t* ring, int it, int* tile, volatile int* abort_flag,
+                      int32_t* status, int kind) {
+  const int j = it % SCHED;
+  const uint32_t want = (uint32_t)it + 1u;
+  uint64_t v = ring[j];
+  bool ok = (uint32_t)(v >> 32) == want;
+  if (!ok) {
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t k = 1;; ++k) {
+      v = ring[j];
+      const uint32_t tag = (uint32_t)(v >> 32);
+      if (tag == want) {
+        ok = true;
+        break;
+      }
+      if (tag > want) break;  // overwritten: cannot happen within the bound
+      if ((k & 31u) == 0 && (*abort_flag || globaltimer() - t0 > kWaitLimitNs)) break;
+    }
+  }
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok) {
+    raise_abort(abort_flag, status, kind);
+    return false;
+  }
+  *tile = __shfl_sync(0xffffffffu, (int)(uint32_t)v, 0);
+  return true;
 }
 
 // Self-test of the bounded wait above, on one CTA of two warps. Warp 0 waits
@@ -239,7 +313,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile uint64_t* ring = tempty + 2;  // [SCHED] tile-index ring
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2 + SCHED);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -256,6 +331,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
       mbar_init(&tfull[a], 1);   // one multicast commit per finished accumulator
       mbar_init(&tempty[a], 2 * Op<KIND>::EPI_WARPS);  // leader: epilogue warps of both CTAs
     }
+    for (int j = 0; j < SCHED; ++j) ring[j] = 0;  // no tag yet
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -274,6 +350,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
   // set-up above overlaps the previous kernel's tail; global memory only from here
   pdl_wait();
   pdl_trigger();
+  if (blockIdx.x == 0 && threadIdx.x == 0 && args.next_ctr != nullptr) *args.next_ctr = 0;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -282,7 +359,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = cluster; ok && tile < num_tiles; tile += num_clusters) {
+    // The leader fetches two tiles ahead: once the first loads of its it-th
+    // tile are issued it publishes the following tile (fetched a tile
+    // earlier, so the atomic's latency has passed) and fetches the one after
+    // that. The peer's producer then finds its next tile published when it
+    // needs it. A fetch left unpublished when the loop ends came after the
+    // index that ended it, so it is past the last tile too.
+    auto fetch = [&](int fallback) {
+      int v = fallback;
+      if (rank == 0 && lane == 0 && args.tile_ctr != nullptr)
+        v = num_clusters + atomicAdd(args.tile_ctr, 1);
+      return v;
+    };
+    int tile = cluster;
+    int next = fetch(cluster + num_clusters);
+    for (int it = 0; ok && tile < num_tiles; ++it) {
+      int after = 0;
       // A block b of this CTA: rows m0 + b * 2 * BM .. + BM (the pair's
       // 256-row MMA b takes block b of both CTAs)
       const int m0 = (tile / args.tiles_n) * TILE_ROWS + (int)rank * BM;
@@ -325,6 +417,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
           stage = 0;
           phase ^= 1u;
         }
+        if (kb == 0 && rank == 0) {  // after this tile's first loads are on their way
+          next = __shfl_sync(0xffffffffu, next, 0);
+          ring_publish(ring, it, next);
+          after = fetch(next + num_clusters);
+        }
+      }
+      if (!ok) break;
+      if (rank == 0) {
+        tile = next;
+        next = after;
+      } else if (!ring_next(ring, it, &tile, abort_flag, args.status, KIND)) {
+        ok = false;
+        break;
       }
     }
     // Wait until the last stages are released, so that no MMA-completion
@@ -343,9 +448,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
           F8 ? idesc_e4m3(2 * BM, BN) : idesc_bf16(2 * BM, BN, Op<KIND>::A_MN, Op<KIND>::B_MN);
       int stage = 0;
       uint32_t phase = 0;
-      int it = 0;
       bool ok = true;
-      for (int tile = cluster; ok && tile < num_tiles; tile += num_clusters, ++it) {
+      int tile = cluster;
+      for (int it = 0; ok && tile < num_tiles; ++it) {
         const int acc = it % ACC;
         const uint32_t acc_phase = (it / ACC) & 1;
         if (!warp_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status, KIND)) break;
@@ -386,6 +491,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
         if (!ok) break;
         if (lane == 0) umma_commit_pair(&tfull[acc], 0x3);  // both halves of the tile ready
         __syncwarp();
+        if (!ring_next(ring, it, &tile, abort_flag, args.status, KIND)) break;
       }
     }
   } else {
@@ -397,7 +503,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
     const int e = warp - 2;   // staging slot
     const int half = e / 4;   // which part of the tile's columns
     const int c_begin = half * CPW;
-    int it = 0;
     uint32_t store_ctr = 0;
     // the forward's E is a write-once stream larger than L2: evict it first
     const uint64_t store_policy = IS_FWD ? policy_evict_first() : 0;
@@ -427,7 +532,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
         }
       }
     }
-    for (int tile = cluster; tile < num_tiles; tile += num_clusters, ++it) {
+    int tile = cluster;
+    for (int it = 0; tile < num_tiles; ++it) {
       const int acc = it % ACC;
       const uint32_t acc_phase = (it / ACC) & 1;
       const int m_blk = tile / args.tiles_n, n_blk = tile % args.tiles_n;
@@ -611,6 +717,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<KIND>(),
         }
         if (IS_FWD && row_ok) args.rowsum[(size_t)(n_blk * HALVES + half) * args.M + row] = s_tile;
       }
+      if (!ring_next(ring, it, &tile, abort_flag, args.status, KIND)) break;
     }
     if (lane == 0) bulk_wait<0>();
     __syncwarp();

@@ -37,6 +37,10 @@ struct GemmArgs {
   int32_t V;
   const int32_t* vocab_pos;  // [V] (dW) rows with -1 are set to +0.0 by the epilogue warps
   int32_t* status;  // dev_status + 8 (error word, detail word)
+  // dynamic tile schedule: this launch's tile counter (zero when it starts),
+  // and a counter it sets to zero for the GEMM that follows it (or null)
+  int32_t* tile_ctr;
+  int32_t* next_ctr;
 };
 
 // KIND_FWD8: the forward on e4m3 operands (x and W_C quantized per tensor).

@@ -205,6 +205,12 @@ SS_DEV void cluster_sync() {
                    "memory");
 }
 
+// 64-bit store to shared memory given by its shared::cluster address (may be
+// the peer's).
+SS_DEV void st_shared_cluster_u64(uint32_t cluster_addr, uint64_t v) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(cluster_addr), "l"(v) : "memory");
+}
+
 // Arrive on an mbarrier given by its shared::cluster address (may be the peer's).
 SS_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)

@@ -202,7 +202,7 @@ Layout layout(int64_t T, int32_t d, int32_t V, int32_t P) {
   L.rscale = take((size_t)T * 4, 256);
   L.loss_rows = take((size_t)T * 4, 256);
   L.fix_list = take((size_t)T * 4, 256);
-  L.fix_count = take(16, 256);
+  L.fix_count = take(kCounterWords * 4, 256);
   L.partials = take((size_t)kRowPartials * sizeof(double2), 256);
   L.w_c = take((size_t)P * d * 2, 1024);
   L.u = take((size_t)T * L.ldz * 2, 1024);
@@ -320,7 +320,7 @@ static ss_status forward_impl(const ss_bf16* x, const ss_bf16* lm_head,
   uint8_t* x8 = ws + L.x8;
   uint8_t* w8 = ws + L.w8;
   float* qscale = reinterpret_cast<float*>(ws + L.qscale);
-  uint32_t* amax = reinterpret_cast<uint32_t*>(fix_count + 1);  // zeroed with fix_count
+  uint32_t* amax = reinterpret_cast<uint32_t*>(fix_count + kWordAmax);  // zeroed with fix_count
   if (e4m3) {
     ra.x8 = x8;
     ra.w8 = w8;
@@ -328,7 +328,8 @@ static ss_status forward_impl(const ss_bf16* x, const ss_bf16* lm_head,
   }
 
   SS_LAUNCH("gather", s,
-            launch_gather(lm_head, candidates, P, d, V, w_c, kstatus, fix_count, e4m3 ? 3 : 1, s));
+            launch_gather(lm_head, candidates, P, d, V, w_c, kstatus, fix_count, kCounterWords,
+                          s));
   if (T > 0) {
     CUtensorMap ta, tb, tc;
     ss_status r;
@@ -361,6 +362,7 @@ static ss_status forward_impl(const ss_bf16* x, const ss_bf16* lm_head,
     a.out = u;
     a.ld_out = L.ldz;
     a.status = kstatus;
+    a.tile_ctr = fix_count + kWordFwdTiles;
     const int tiles = a.tiles_m * a.tiles_n;
     SS_LAUNCH_GEMM(e4m3 ? "fwd_gemm_ce_e4m3" : "fwd_gemm_ce", s,
               launch_gemm(kind, ta, tb, tc, a, tiles < pairs[kind] ? tiles : pairs[kind], s));
@@ -497,6 +499,7 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   uint16_t* w_c = reinterpret_cast<uint16_t*>(ws + L.w_c);
   uint16_t* u = reinterpret_cast<uint16_t*>(ws + L.u);
   uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
+  int32_t* counters = reinterpret_cast<int32_t*>(ws + L.fix_count);
   int32_t* kstatus = dev_status + 8;
 
   if (T == 0) {
@@ -528,6 +531,8 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   a.out = dx;
   a.ld_out = d;
   a.status = kstatus;
+  a.tile_ctr = counters + kWordDxTiles;
+  a.next_ctr = counters + kWordDwTiles;
   const int tiles = a.tiles_m * a.tiles_n;
   SS_LAUNCH_GEMM("dx_gemm", s,
             launch_gemm(kdx, ua, wb, dxs, a, tiles < pairs[kdx] ? tiles : pairs[kdx], s));
@@ -546,6 +551,8 @@ ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
   b.grad_loss = grad_loss;
   b.n_valid = n_valid;
   b.status = kstatus;
+  b.tile_ctr = counters + kWordDwTiles;
+  b.next_ctr = counters + kWordDxTiles;
   // every resident pair, even without a tile, so that the zero rows are spread over all SMs
   SS_LAUNCH_GEMM("dw_gemm_scatter", s, launch_gemm(kdw, ua2, xb, ua2, b, pairs[kdw], s));
   return SS_OK;

@@ -73,6 +73,12 @@ struct RowArgs {
 };
 // Most blocks the row pass launches (the size of RowArgs::partials).
 constexpr int kRowPartials = 4096;
+// Words of the workspace's counter block: the row pass's overflow count, the
+// e4m3 amax pair, and the tile counters of the three GEMMs. The forward's
+// gather zeroes all of them; dX zeroes dW's counter and dW zeroes dX's, so
+// that a backward repeated after one forward starts from zero as well.
+constexpr int kWordFixCount = 0, kWordAmax = 1, kWordFwdTiles = 4, kWordDxTiles = 5,
+              kWordDwTiles = 6, kCounterWords = 8;
 cudaError_t launch_rows(const RowArgs& a, cudaStream_t s);
 // Exact recomputation of overflowed rows, then the loss mean (one CTA).
 cudaError_t launch_finalize(const RowArgs& a, cudaStream_t s);

@@ -260,6 +260,30 @@ def test_backward_can_be_repeated():
     assert torch.equal(ce.dW.float(), (2 * dw1.float()).bfloat16().float())
 
 
+def test_backward_repeated_with_more_tiles_than_pairs():
+    """Here both backward GEMMs have several times more tiles than CTA pairs
+    (on 148 SMs: dX 471 and dW 354 tiles of 256 x 256 for 74 pairs), so most
+    tiles come from the dynamic schedule's counters: a second backward after
+    one forward must find its counters reset (dX resets dW's, dW resets dX's)
+    and compute every tile again."""
+    T, d, V, P = 40000, 768, 50304, 30000
+    x, lm, t = random_case(T, d, V, P, 31)
+    ce = capi.SampledCE(T, d, V, P)
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    lt = torch.from_numpy(lm.view(np.int16)).view(torch.bfloat16).cuda()
+    ce.build(torch.from_numpy(t).cuda(), 5)
+    ce.forward(xt, lt)
+    ce.backward()
+    dx1, dw1 = ce.dx.clone(), ce.dW.clone()
+    for g in (2.0, 0.5):
+        ce.grad_loss.fill_(g)
+        ce.backward()
+        torch.cuda.synchronize()
+        assert ce.status()[8] == 0
+        assert torch.equal(ce.dx.float(), (g * dx1.float()).bfloat16().float())
+        assert torch.equal(ce.dW.float(), (g * dw1.float()).bfloat16().float())
+
+
 def test_deterministic():
     x, lm, t = random_case(1000, 200, 5003, 3000, 13)
     a = run_path(x, lm, t, 3000, 17)
