@@ -215,8 +215,11 @@ SS_API ss_status ss_quantize_e4m3(const ss_bf16* src, int64_t n, uint8_t* dst, f
  * dW_C = (g/n) E'^T @ x'.
  * In:  grad_loss [1] float32 (device); candidates, vocab_pos as above; n_valid
  *      from ss_ce_forward; the workspace the forward used (it holds the x' rows).
- * Out: dx [T, d], dW [V, d] (fully written). The workspace is only read, so
- *      the backward may be repeated (for another grad_loss) after one forward. */
+ * Out: dx [T, d], dW [V, d] (fully written). Of the workspace the backward
+ *      writes only the two GEMMs' tile counters (each GEMM hands its output
+ *      tiles to CTA pairs through one; dX resets dW's and dW resets dX's), so
+ *      the backward may be repeated (for another grad_loss) after one forward;
+ *      as with every call, one workspace serves one stream at a time. */
 SS_API ss_status ss_ce_backward(const float* grad_loss, const int32_t* candidates,
                          const int32_t* vocab_pos, const int32_t* n_valid, int64_t T,
                          int32_t d, int32_t V, int32_t P, ss_bf16* dx, ss_bf16* dW,
