@@ -1,4 +1,5 @@
-"""GPU: many steps in a row, and two independent steps on two streams at once.
+"""GPU: many steps in a row, two independent steps on two streams at once, and
+steps while another stream's kernel holds SMs.
 
 compute-sanitizer's race checker is not available here, so these look for
 races the way a long training run would meet them: results that change from
@@ -7,7 +8,10 @@ times per launch and across launches), or that depend on what another
 stream runs at the same time (the workspace entry points keep no state
 between calls, so two workspaces on two streams must not interfere; the
 allocation-free build is the one exception, with one scratch array per device
-that every call shares, and is not run on two streams here).
+that every call shares, and is not run on two streams here). The GEMMs hand
+their tiles to CTA pairs dynamically, so a pair whose SMs another kernel
+still holds takes fewer tiles: which pair computes which tile then changes
+from step to step, and the results must not.
 """
 
 import hashlib
@@ -78,3 +82,43 @@ def test_two_streams_match_one_stream(precision):
     for (ce, _), want in zip(sets, ref):
         assert ce.status()[8] == 0
         assert _digest(ce) == want
+
+
+@pytest.mark.parametrize("precision", ["bf16", "e4m3"])
+def test_steps_with_sms_held_by_another_stream_match(precision):
+    """A bf16 matmul on another stream, started at a varying point of each
+    step, holds SMs while the step's persistent GEMMs start (all three have
+    more tiles than CTA pairs here); every step equals the undisturbed one
+    bit for bit."""
+    T, d, V, P = 16384, 768, 50304, 16384
+    ce = capi.SampledCE(T, d, V, P, precision=precision)
+    x, lm, t = _inputs(T, d, V, 93)
+    ce.step(t, x, lm, 5)
+    torch.cuda.synchronize()
+    outs = (ce.dx, ce.dW, ce.loss, ce.lse, ce.candidates, ce.target_pos)
+    ref = [a.clone() for a in outs]
+    g = torch.Generator(device="cuda").manual_seed(94)
+    a = torch.randn(8192, 8192, device="cuda", dtype=torch.bfloat16, generator=g)
+    side = torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+
+    def hold():
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            a @ a
+
+    rng = np.random.default_rng(95)
+    for _ in range(12):
+        where = int(rng.integers(0, 3))
+        if where == 0:
+            hold()
+        ce.build(t, 5)
+        if where == 1:
+            hold()
+        ce.forward(x, lm)
+        if where == 2:
+            hold()
+        ce.backward()
+        assert all(torch.equal(u, v) for u, v in zip(outs, ref))
+    torch.cuda.synchronize()
+    assert ce.status()[8] == 0
