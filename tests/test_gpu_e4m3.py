@@ -92,6 +92,16 @@ def test_e4m3_small_shapes_match_oracle(T, d, V, P, seed, grad):
     assert abs(g["loss"] - ob["loss"]) > abs(g["loss"] - o["loss"])
 
 
+def test_e4m3_one_k_block_forward_with_many_tiles():
+    """d = 128: one 128-deep K block of e4m3 codes per forward tile (the
+    dynamic tile schedule's producer furthest ahead), 1024 tiles."""
+    T, d, V, P, seed = 8192, 128, 20000, 8192, 44
+    x, lm, t = wl.make_inputs(T, d, V, 1.1, 0.05, seed)
+    g = run_path(x, lm, t, P, 17, precision="e4m3")
+    o = _e4m3_oracle(x, lm, t, P, 17)
+    compare_full(g, o, t)
+
+
 def test_e4m3_rows_with_huge_loss_are_recomputed_exactly():
     T, d, V, P, seed = 300, 64, 1000, 384, 21
     x, lm, t = wl.make_inputs(T, d, V, 1.1, 0.05, seed)

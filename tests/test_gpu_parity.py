@@ -176,6 +176,23 @@ def test_edge_shapes_match_oracle(kind):
         assert np.max(np.abs(wl.bits_to_f64(g["dx_bits"]))) <= 1e-6
 
 
+@pytest.mark.parametrize("T,d,V,P,seed", [
+    (8192, 64, 20000, 8192, 41),   # forward: d = 64, one K block; 1024 tiles
+    (32768, 768, 64, 64, 42),      # dX: K = P = 64, one K block; 384 tiles
+    (64, 768, 50304, 40000, 43),   # dW: K = T = 64, one K block; 471 tiles
+])
+def test_one_k_block_gemms_with_many_tiles_compared_in_full(T, d, V, P, seed):
+    """A tile with a single K block lets the dynamic tile schedule's producer
+    run furthest ahead of the warps that read its tile ring (the ring's size
+    is set by that case); each shape gives one GEMM a single K block and more
+    tiles than CTA pairs, compared in full."""
+    x, lm, t = random_case(T, d, V, P, seed)
+    off = (seed * 7919) % V
+    g = run_path(x, lm, t, P, off)
+    o = oracle_run(x, lm, t, P, off)
+    compare_full(g, o, t)
+
+
 def test_tiny_workload_matches_oracle():
     w = wl.WORKLOADS["tiny"]
     x, lm, t = wl.workload_inputs(w)
